@@ -1,0 +1,196 @@
+"""Thin Python binding of ``liblightning.so`` (argument marshalling only).
+
+Each function takes torch tensors, checks that they are contiguous CUDA
+tensors of the expected dtype, and passes their data pointers, sizes and the
+current CUDA stream to the C entry point of the same name.  Every step of the
+computation runs in the library's kernels; there is no Python or CPU path, and
+a missing or unloadable library raises ``LightningLibraryError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA = 0, 1, 2, 3
+LA_ERR_DEVICE_TIMEOUT, LA_ERR_DEVICE_RANGE = 4, 5
+LA_FP32, LA_BF16, LA_OUT_RMSNORM, LA_WRITE_STATE = 0, 1, 2, 4
+LA_MAX_VARLEN_SEQS = 1024
+
+
+class LightningLibraryError(RuntimeError):
+    """The CUDA library is missing or could not be loaded."""
+
+
+class LightningError(RuntimeError):
+    """A library call returned a status other than LA_OK."""
+
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: {text} ({status})")
+        self.status = status
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library with argument types declared (loads it on first use)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = os.environ.get("LA_LIBRARY", _build.LIB)
+    if not os.path.exists(path):
+        raise LightningLibraryError(
+            f"{path} is missing: build it with `python -m long_context_04_b200.build`")
+    try:
+        L = ctypes.CDLL(path)
+    except OSError as e:  # pragma: no cover - depends on the machine
+        raise LightningLibraryError(f"cannot load {path}: {e}") from e
+    vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+    ip = ctypes.POINTER(ctypes.c_int32)
+    L.la_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ip, i32, u32, vp, vp]
+    L.la_prefill.restype = i32
+    L.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, u32, vp]
+    L.la_decode_step.restype = i32
+    L.la_state_out.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp]
+    L.la_state_out.restype = i32
+    L.la_status_string.argtypes = [i32]
+    L.la_status_string.restype = ctypes.c_char_p
+    L.la_get_device_status.argtypes = [vp]
+    L.la_get_device_status.restype = i32
+    L.la_version.argtypes = []
+    L.la_version.restype = i32
+    _LIB = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().la_status_string(status).decode()
+
+
+def _check(fn: str, status: int):
+    if status != LA_OK:
+        raise LightningError(fn, status, status_string(status))
+
+
+def _stream_ptr(stream) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _flags_for(dtype) -> int:
+    if dtype == torch.bfloat16:
+        return LA_BF16
+    if dtype == torch.float32:
+        return LA_FP32
+    raise ValueError(f"unsupported dtype {dtype}: bf16 or fp32")
+
+
+def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
+            return_state: bool = False, state_out=None, out=None, stream=None):
+    """Causal lightning attention over a batch (length > 1 path).
+
+    ``q, k, v``: ``[B, N, H, D]`` or packed ``[T, H, D]`` (then ``cu_seqlens``,
+    a host sequence of S+1 ints, gives the boundaries).  Returns ``o`` of the
+    same shape, or ``(o, state)`` with ``return_state`` (state ``[S, H, D, D]``
+    fp32, the final K^T V of each sequence).
+    """
+    _need(q, "q")
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+        if t.shape != q.shape:
+            raise ValueError("q, k, v must have one shape")
+    flags = _flags_for(q.dtype)
+    if q.dim() == 4:
+        B, N, H, D = q.shape
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens needs packed [T, H, D] inputs")
+        S = B
+    elif q.dim() == 3:
+        T, H, D = q.shape
+        B, N = 1, T
+        S = 1 if cu_seqlens is None else len(cu_seqlens) - 1
+    else:
+        raise ValueError("q must be [B, N, H, D] or [T, H, D]")
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype)
+    st = state_out
+    if return_state and st is None:
+        st = torch.empty((S, H, D, D), dtype=torch.float32, device=q.device)
+    if st is not None:
+        _need(st, "state_out", torch.float32)
+        flags |= LA_WRITE_STATE
+    if rmsnorm:
+        flags |= LA_OUT_RMSNORM
+    cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    rc = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, D, beta, cu_ptr,
+                          0 if cu is None else len(cu) - 1, flags, _ptr(st), _stream_ptr(stream))
+    _check("la_prefill", rc)
+    return (out, st) if (return_state or state_out is not None) else out
+
+
+def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None):
+    """One token per sequence: ``state += k v^T`` in place, returns ``o = q^T state``.
+
+    ``q, k, v``: ``[B, H, D]``; ``state``: ``[B, H, D, D]`` fp32.
+    """
+    _need(q, "q")
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+        if t.shape != q.shape:
+            raise ValueError("q, k, v must have one shape")
+    _need(state, "state", torch.float32)
+    B, H, D = q.shape
+    if tuple(state.shape) != (B, H, D, D):
+        raise ValueError("state must be [B, H, D, D]")
+    flags = _flags_for(q.dtype) | (LA_OUT_RMSNORM if rmsnorm else 0)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype)
+    rc = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H, D, flags,
+                              _stream_ptr(stream))
+    _check("la_decode_step", rc)
+    return out
+
+
+def state_out(state_ws, state_dst, seq_to_slot=None, *, stream=None):
+    """``state_dst[slot(s)] = state_ws[s]`` (slot = ``seq_to_slot[s]``, a CUDA int32 tensor)."""
+    _need(state_ws, "state_ws", torch.float32)
+    _need(state_dst, "state_dst", torch.float32)
+    S, H, D, _ = state_ws.shape
+    if seq_to_slot is not None:
+        _need(seq_to_slot, "seq_to_slot", torch.int32)
+    rc = lib().la_state_out(_ptr(state_ws), _ptr(state_dst), S, H, D, _ptr(seq_to_slot),
+                            state_dst.shape[0], _stream_ptr(stream))
+    _check("la_state_out", rc)
+    return state_dst
+
+
+def device_status(stream=None) -> int:
+    """Synchronise ``stream`` and return (and clear) the device status word."""
+    return lib().la_get_device_status(_stream_ptr(stream))
+
+
+def version() -> int:
+    return lib().la_version()

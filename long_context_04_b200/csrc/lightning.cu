@@ -1,0 +1,256 @@
+// liblightning.so: the C ABI declared in include/lightning_attention.h.
+//
+// Host side only: argument validation, the sequence table, TMA tensor maps and
+// kernel launches.  Every step of the computation runs in the kernels of
+// prefill_tc.cuh (bf16, tcgen05), prefill_simt.cuh (fp32), decode.cuh.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <numeric>
+#include <vector>
+
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+
+namespace {
+
+using la::PrefillTcParams;
+using la::SeqTable;
+
+constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cuTensorMapEncodeTiled, fetched through the runtime so that the library does
+// not link libcuda directly.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [T][H*D] bf16 viewed as a 2-D tensor; boxes of 64 columns x beta rows, 128-B swizzle.
+bool make_map(CUtensorMap *map, const void *base, long long T, int H, int D, int beta) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)H * D, (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)H * D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)beta};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int BETA, int D>
+la_status launch_tc(const PrefillTcParams &p, int units, cudaStream_t stream) {
+    using C = la::TcCfg<BETA, D>;
+    auto kern = la::prefill_tc_kernel<BETA, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)units);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C::NVS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+template <int BETA, int D>
+la_status launch_simt(const float *q, const float *k, const float *v, float *o, float *state,
+                      int H, int rmsnorm, const SeqTable &seqs, int S, cudaStream_t stream) {
+    using C = la::SimtCfg<BETA, D>;
+    auto kern = la::prefill_simt_kernel<BETA, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    kern<<<S * H, C::THREADS, C::SMEM_BYTES, stream>>>(q, k, v, o, state, H, rmsnorm, seqs);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA";
+        case LA_ERR_DEVICE_TIMEOUT: return "LA_ERR_DEVICE_TIMEOUT";
+        case LA_ERR_DEVICE_RANGE: return "LA_ERR_DEVICE_RANGE";
+    }
+    return "LA_ERR_UNKNOWN";
+}
+
+int la_version(void) { return 100; }
+
+la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B, int H, int N,
+                     int D, int beta, const int32_t *cu_seqlens, int num_seqs, unsigned flags,
+                     float *state_ws, void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const unsigned known = LA_BF16 | LA_OUT_RMSNORM | LA_WRITE_STATE;
+    if (flags & ~known) return LA_ERR_INVALID_ARG;
+    if (H < 1 || N < 0 || B < 1) return LA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LA_ERR_INVALID_ARG;
+    const bool want_state = (flags & LA_WRITE_STATE) != 0;
+    if (want_state && (state_ws == nullptr || !aligned16(state_ws))) return LA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+    if (beta != 64 && beta != 128) return LA_ERR_UNSUPPORTED;
+
+    // Sequence table (host-validated).
+    SeqTable seqs;
+    std::memset(&seqs, 0, sizeof seqs);
+    long long T = 0;
+    int S = 0;
+    if (cu_seqlens != nullptr) {
+        if (B != 1) return LA_ERR_INVALID_ARG;
+        if (num_seqs < 1) return LA_ERR_INVALID_ARG;
+        if (num_seqs > LA_MAX_VARLEN_SEQS) return LA_ERR_UNSUPPORTED;
+        if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != N) return LA_ERR_INVALID_ARG;
+        for (int s = 0; s < num_seqs; ++s)
+            if (cu_seqlens[s + 1] < cu_seqlens[s]) return LA_ERR_INVALID_ARG;
+        S = num_seqs;
+        T = N;
+        std::vector<int> order(S);
+        std::iota(order.begin(), order.end(), 0);
+        std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+            return cu_seqlens[a + 1] - cu_seqlens[a] > cu_seqlens[b + 1] - cu_seqlens[b];
+        });
+        seqs.varlen = 1;
+        for (int r = 0; r < S; ++r) {
+            const int s = order[r];
+            seqs.seq_start[r] = cu_seqlens[s];
+            seqs.seq_len[r] = cu_seqlens[s + 1] - cu_seqlens[s];
+            seqs.seq_id[r] = s;
+        }
+    } else {
+        S = B;
+        T = (long long)B * N;
+        seqs.varlen = 0;
+        seqs.N = N;
+    }
+    if (T >= (1ll << 31) || (long long)S * H * 2 >= (1ll << 31)) return LA_ERR_UNSUPPORTED;
+    if (S == 0 || H == 0) return LA_OK;
+
+    const int rms = (flags & LA_OUT_RMSNORM) ? 1 : 0;
+    float *state = want_state ? state_ws : nullptr;
+
+    if (flags & LA_BF16) {
+        if (T == 0 && !want_state) return LA_OK;
+        PrefillTcParams p;
+        std::memset(&p, 0, sizeof p);
+        const long long Tm = T > 0 ? T : 1;  // a tensor map needs a non-empty extent
+        if (!make_map(&p.tmap_q, q, Tm, H, D, beta) || !make_map(&p.tmap_k, k, Tm, H, D, beta) ||
+            !make_map(&p.tmap_v, v, Tm, H, D, beta))
+            return LA_ERR_CUDA;
+        p.o = static_cast<__nv_bfloat16 *>(o);
+        p.state = state;
+        p.H = H;
+        p.rmsnorm = rms;
+        p.timeout_ns = kWaitLimitNs;
+        p.seqs = seqs;
+        const int units = S * H * (D / 64);
+        if (beta == 128 && D == 128) return launch_tc<128, 128>(p, units, stream);
+        if (beta == 64 && D == 128) return launch_tc<64, 128>(p, units, stream);
+        if (beta == 128 && D == 64) return launch_tc<128, 64>(p, units, stream);
+        return launch_tc<64, 64>(p, units, stream);
+    }
+    const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
+                *vf = static_cast<const float *>(v);
+    float *of = static_cast<float *>(o);
+    if (beta == 128 && D == 128) return launch_simt<128, 128>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
+    if (beta == 64 && D == 128) return launch_simt<64, 128>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
+    if (beta == 128 && D == 64) return launch_simt<128, 64>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
+    return launch_simt<64, 64>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, float *state, void *o, int B,
+                         int H, int D, unsigned flags, void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const unsigned known = LA_BF16 | LA_OUT_RMSNORM;
+    if (flags & ~known) return LA_ERR_INVALID_ARG;
+    if (B < 0 || H < 1) return LA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !state) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+        return LA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+    if ((long long)B * H >= (1ll << 31)) return LA_ERR_UNSUPPORTED;
+    if (B == 0) return LA_OK;
+    const int rms = (flags & LA_OUT_RMSNORM) ? 1 : 0;
+    const unsigned grid = (unsigned)(B * H);
+    if (flags & LA_BF16) {
+        using T = __nv_bfloat16;
+        if (D == 128)
+            la::decode_step_kernel<128, T><<<grid, 256, 0, stream>>>(
+                (const T *)q, (const T *)k, (const T *)v, state, (T *)o, rms);
+        else
+            la::decode_step_kernel<64, T><<<grid, 256, 0, stream>>>(
+                (const T *)q, (const T *)k, (const T *)v, state, (T *)o, rms);
+    } else {
+        if (D == 128)
+            la::decode_step_kernel<128, float><<<grid, 256, 0, stream>>>(
+                (const float *)q, (const float *)k, (const float *)v, state, (float *)o, rms);
+        else
+            la::decode_step_kernel<64, float><<<grid, 256, 0, stream>>>(
+                (const float *)q, (const float *)k, (const float *)v, state, (float *)o, rms);
+    }
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_state_out(const float *state_ws, float *state_dst, int S, int H, int D,
+                       const int32_t *seq_to_slot, int num_slots, void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (S < 0 || H < 1 || num_slots < 0) return LA_ERR_INVALID_ARG;
+    if (!state_ws || !state_dst) return LA_ERR_INVALID_ARG;
+    if (!aligned16(state_ws) || !aligned16(state_dst)) return LA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+    if (seq_to_slot == nullptr && S > num_slots) return LA_ERR_INVALID_ARG;
+    if ((long long)S * H >= (1ll << 31)) return LA_ERR_UNSUPPORTED;
+    if (S == 0) return LA_OK;
+    la::state_copy_kernel<<<(unsigned)(S * H), 256, 0, stream>>>(
+        reinterpret_cast<const float4 *>(state_ws), reinterpret_cast<float4 *>(state_dst),
+        seq_to_slot, H, D * D / 4, num_slots);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_get_device_status(void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return LA_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, la::g_device_status, sizeof word) != cudaSuccess)
+        return LA_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(la::g_device_status, &zero, sizeof zero) != cudaSuccess)
+        return LA_ERR_CUDA;
+    if (word == la::DEV_TIMEOUT) return LA_ERR_DEVICE_TIMEOUT;
+    if (word == la::DEV_RANGE) return LA_ERR_DEVICE_RANGE;
+    return LA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,498 @@
+// Lightning-attention prefill for bf16 inputs on sm_100a: TMA + tcgen05 + TMEM.
+//
+// Method (MiniMax-01, "Scaling Foundation Models with Lightning Attention";
+// CSDN digest section 2.1, mizuki blog appendix "key concepts"): for every
+// block b of BETA tokens of one sequence and one head,
+//     O_b = [(Q_b K_b^T) (.) M] V_b + Q_b KV,     KV += K_b^T V_b,
+// with the causal 0/1 mask M (j <= i) and KV reset at each sequence start,
+// followed by an optional RMSNorm of each output row over the head dim.
+//
+// One CTA owns one work unit (sequence, head, 64-column slice of V/O).  With
+// D = 128 the two slices of a (sequence, head) form a 2-CTA cluster: both
+// recompute S = Q_b K_b^T (the second reads Q/K from L2) and exchange per-row
+// sums of squares through distributed shared memory for the RMSNorm.  All
+// four block contractions run on the tensor cores with fp32 accumulators in
+// TMEM; the D x 64 fp32 state lives in TMEM for the whole sequence.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: Q_b, K_b (D columns) and V_b (64 columns) into a
+//               ring of NST shared-memory stages.
+//   warp 1      TMEM owner and MMA issuer (lane 0 issues; the warp zeroes the
+//               V rows past a sequence end before they enter K^T V).
+//   warps 2..5  epilogue: S -> masked bf16 P (shared memory), fp32 state ->
+//               bf16 snapshot for the next block's Q_b KV, O -> (RMSNorm) ->
+//               bf16 global store, final state -> fp32 global store.
+// Per block the MMA issue order is: S_{b+1} (look-ahead), O_b = P_b V_b,
+// O_b += Q_b snap(KV_{<b}), KV += K_b^T V_b; one commit then releases the
+// stage, P, the O buffer and the state to the other roles.
+// Every wait is bounded (see mbar_wait); on a timeout the CTA records
+// DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include "la_device.cuh"
+#include "../../include/lightning_attention.h"
+
+namespace la {
+
+// Sequences of one call.  Uniform batches (varlen = 0) use start = r * N and
+// length N.  Packed batches list their sequences longest first, so that the
+// hardware block scheduler, which starts CTAs in index order, hands out the
+// longest chains first.
+struct SeqTable {
+    int varlen;
+    int N;
+    int seq_start[LA_MAX_VARLEN_SEQS];
+    int seq_len[LA_MAX_VARLEN_SEQS];
+    int seq_id[LA_MAX_VARLEN_SEQS];  // index of the sequence in the caller's order
+
+    __device__ __forceinline__ void get(int r, int &start, int &len, int &sid) const {
+        if (varlen) {
+            start = seq_start[r];
+            len = seq_len[r];
+            sid = seq_id[r];
+        } else {
+            start = r * N;
+            len = N;
+            sid = r;
+        }
+    }
+};
+
+struct PrefillTcParams {
+    CUtensorMap tmap_q;  // [T][H*D] bf16, box 64 x BETA, 128-byte swizzle
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    __nv_bfloat16 *o;
+    float *state;        // [S][H][D][D] or nullptr
+    int H;
+    int rmsnorm;
+    unsigned long long timeout_ns;
+    SeqTable seqs;
+};
+
+template <int BETA, int D>
+struct TcCfg {
+    static constexpr int NVS = D / 64;          // CTAs per (sequence, head)
+    static constexpr int DV = 64;               // output columns per CTA
+    static constexpr int DB = D / 64;           // 64-column tiles in Q or K
+    static constexpr int BOX = BETA * 128;      // one 64-column tile of BETA rows (bytes)
+    static constexpr int STAGE = (2 * DB + 1) * BOX;
+    static constexpr int P_BYTES = (BETA / 64) * BOX;
+    static constexpr int SNAP_BYTES = D * 128;
+    static constexpr int SMEM_LIMIT = 227 * 1024;
+    static constexpr int MISC = 2048;
+    static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - P_BYTES - SNAP_BYTES - MISC) / STAGE;
+    static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
+    static_assert(NST >= 2, "shared memory budget");
+    static constexpr int OFF_P = NST * STAGE;
+    static constexpr int OFF_SNAP = OFF_P + P_BYTES;
+    static constexpr int OFF_MISC = OFF_SNAP + SNAP_BYTES;
+    // At least 120 KB so that no two CTAs share an SM: each allocates all 512
+    // TMEM columns, and a second resident CTA would block in tcgen05.alloc.
+    static constexpr int SMEM_USED = 1024 + OFF_MISC + MISC;
+    static constexpr int SMEM_BYTES = SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
+    // TMEM columns
+    static constexpr int TM_S = 0;              // two BETA-column S buffers
+    static constexpr int TM_O = 2 * BETA;       // two 64-column O buffers
+    static constexpr int TM_KV = 2 * BETA + 128;
+    static constexpr int TMEM_COLS = 512;
+    static_assert(TM_KV + 64 <= TMEM_COLS, "TMEM budget");
+    static constexpr int EPI_THREADS = 128;
+    static constexpr int THREADS = 64 + EPI_THREADS;
+    static constexpr uint32_t ID_S = idesc_bf16_f32(BETA, BETA, 0, 0);
+    static constexpr uint32_t ID_PV = idesc_bf16_f32(BETA, 64, 0, 1);
+    static constexpr uint32_t ID_QKV = idesc_bf16_f32(BETA, 64, 0, 1);
+    static constexpr uint32_t ID_KV = idesc_bf16_f32(D, 64, 1, 1);
+};
+
+// Barriers and small shared state, placed after the tiles.
+template <int NST, int BETA>
+struct TcMisc {
+    uint64_t full[NST];
+    uint64_t empty[NST];
+    uint64_t s_full[2];
+    uint64_t o_full[2];
+    uint64_t o_free[2];
+    uint64_t ss_full[2];
+    uint64_t p_ready;
+    uint64_t p_free;
+    uint64_t kv_full;
+    uint64_t snap_ready;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    float ss_in[2][BETA];
+};
+
+template <int BETA, int D>
+__global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
+    prefill_tc_kernel(const __grid_constant__ PrefillTcParams p) {
+    using C = TcCfg<BETA, D>;
+    using Misc = TcMisc<C::NST, BETA>;
+    static_assert(sizeof(Misc) <= C::MISC, "misc area");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    Misc *m = reinterpret_cast<Misc *>(smem + C::OFF_MISC);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int unit = blockIdx.x;
+    const int vs = unit % C::NVS;
+    const int rh = unit / C::NVS;
+    const int h = rh % p.H;
+    const int rank = rh / p.H;
+    int seq_start, seq_len, sid;
+    p.seqs.get(rank, seq_start, seq_len, sid);
+    const int nb = (seq_len + BETA - 1) / BETA;
+    const uint32_t partner = (uint32_t)(vs ^ 1);
+    const uint64_t tlimit = p.timeout_ns;
+    volatile int *abort_flag = &m->abort_flag;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&m->s_full[i], 1);
+            mbar_init(&m->o_full[i], 1);
+            mbar_init(&m->o_free[i], C::EPI_THREADS);
+            mbar_init(&m->ss_full[i], C::EPI_THREADS);
+        }
+        mbar_init(&m->p_ready, C::EPI_THREADS);
+        mbar_init(&m->p_free, 1);
+        mbar_init(&m->kv_full, 1);
+        mbar_init(&m->snap_ready, C::EPI_THREADS);
+        mbar_init(&m->drain, 1);
+        m->abort_flag = 0;
+        fence_mbarrier_init_cluster();
+        tma_prefetch_desc(&p.tmap_q);
+        tma_prefetch_desc(&p.tmap_k);
+        tma_prefetch_desc(&p.tmap_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(&m->tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (C::NVS > 1) cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem = m->tmem_base;
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        record_fault(DEV_TIMEOUT);
+    };
+    auto stage_addr = [&](int st) { return sbase + (uint32_t)(st * C::STAGE); };
+    // Warp-uniform bounded wait: every lane polls (and so acquires), and the
+    // warp proceeds only if all lanes saw the phase complete, so that the
+    // warp-collective tcgen05 instructions after it stay converged.
+    auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, tlimit)) != 0;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int issued = 0;
+        if (lane == 0) {
+            for (int b = 0; b < nb; ++b) {
+                const int st = b % C::NST;
+                const uint32_t ph = (uint32_t)((b / C::NST) & 1);
+                if (!mbar_wait(&m->empty[st], ph ^ 1u, abort_flag, tlimit)) {
+                    fail();
+                    break;
+                }
+                mbar_arrive_expect_tx(&m->full[st], (uint32_t)C::STAGE);
+                const int row = seq_start + b * BETA;
+                const uint32_t sa = stage_addr(st);
+                for (int c = 0; c < C::DB; ++c) {
+                    tma_load_2d(sa + c * C::BOX, &p.tmap_q, h * D + 64 * c, row, &m->full[st]);
+                    tma_load_2d(sa + (C::DB + c) * C::BOX, &p.tmap_k, h * D + 64 * c, row,
+                                &m->full[st]);
+                }
+                tma_load_2d(sa + 2 * C::DB * C::BOX, &p.tmap_v, h * D + 64 * vs, row, &m->full[st]);
+                ++issued;
+            }
+            // Drain: the last NST issued loads must have landed before the CTA exits.
+            for (int b = (issued > C::NST ? issued - C::NST : 0); b < issued; ++b)
+                mbar_wait(&m->full[b % C::NST], (uint32_t)((b / C::NST) & 1), nullptr, tlimit);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        bool any_issued = false;
+        const uint32_t tS[2] = {tmem + C::TM_S, tmem + C::TM_S + BETA};
+        const uint32_t tO[2] = {tmem + C::TM_O, tmem + C::TM_O + 64};
+        const uint32_t tKV = tmem + C::TM_KV;
+        const uint32_t sP = sbase + C::OFF_P, sSnap = sbase + C::OFF_SNAP;
+
+        // Wait for block j's tiles, zero the V rows past the sequence end, issue S_j.
+        auto stage_in = [&](int j) -> bool {
+            const int st = j % C::NST;
+            if (!wwait(&m->full[st], (uint32_t)((j / C::NST) & 1))) return false;
+            const int nv = min(BETA, seq_len - j * BETA);
+            if (nv < BETA) {
+                const uint32_t v0 = stage_addr(st) + 2 * C::DB * C::BOX;
+                for (uint32_t a = v0 + nv * 128 + lane * 16; a < v0 + C::BOX; a += 32 * 16)
+                    st_shared_v4(a, 0u, 0u, 0u, 0u);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sa = stage_addr(st);
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (uint32_t)((ks >> 2) * C::BOX + (ks & 3) * 32);
+                    mma_bf16_ss(tS[j & 1], desc_kmajor_sw128(sa + off),
+                                desc_kmajor_sw128(sa + C::DB * C::BOX + off), C::ID_S,
+                                ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&m->s_full[j & 1]);
+            }
+            any_issued = true;
+            __syncwarp();
+            return true;
+        };
+
+        bool ok = nb == 0 || stage_in(0);
+        for (int b = 0; ok && b < nb; ++b) {
+            if (b + 1 < nb && !stage_in(b + 1)) {
+                ok = false;
+                break;
+            }
+            const int st = b % C::NST;
+            const uint32_t sa = stage_addr(st);
+            const uint32_t sV = sa + 2 * C::DB * C::BOX;
+            if (!wwait(&m->p_ready, (uint32_t)(b & 1))) {
+                ok = false;
+                break;
+            }
+            if (b >= 2 && !wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {  // O_b = P_b V_b
+                for (int ks = 0; ks < BETA / 16; ++ks)
+                    mma_bf16_ss(tO[b & 1],
+                                desc_kmajor_sw128(sP + (ks >> 2) * C::BOX + (ks & 3) * 32),
+                                desc_mnmajor_sw128(sV + ks * 2048, C::BOX), C::ID_PV,
+                                ks > 0 ? 1u : 0u);
+            }
+            __syncwarp();
+            if (b >= 1) {
+                if (!wwait(&m->snap_ready, (uint32_t)((b - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {  // O_b += Q_b snap(KV_{<b})
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        mma_bf16_ss(tO[b & 1],
+                                    desc_kmajor_sw128(sa + (ks >> 2) * C::BOX + (ks & 3) * 32),
+                                    desc_mnmajor_sw128(sSnap + ks * 2048, C::BOX), C::ID_QKV, 1u);
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {  // KV += K_b^T V_b
+                for (int ks = 0; ks < BETA / 16; ++ks)
+                    mma_bf16_ss(tKV, desc_mnmajor_sw128(sa + C::DB * C::BOX + ks * 2048, C::BOX),
+                                desc_mnmajor_sw128(sV + ks * 2048, C::BOX), C::ID_KV,
+                                (b > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(&m->o_full[b & 1]);
+                mma_commit(&m->p_free);
+                mma_commit(&m->kv_full);
+                mma_commit(&m->empty[st]);
+            }
+            __syncwarp();
+        }
+        if (!ok) fail();
+        if (any_issued && lane == 0) {  // every issued MMA has finished before TMEM is freed
+            mma_commit(&m->drain);
+            mbar_wait(&m->drain, 0u, nullptr, tlimit);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                    // TMEM lane quadrant of this warp
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int r = BETA == 128 ? 32 * q + lane : 16 * q + lane;   // row of the block
+        const bool r_ok = BETA == 128 || lane < 16;
+        const int i = D == 128 ? 32 * q + lane : 16 * q + lane;      // state row
+        const bool i_ok = D == 128 || lane < 16;
+        const uint32_t sP = sbase + C::OFF_P, sSnap = sbase + C::OFF_SNAP;
+        const size_t o_col = (size_t)h * D + 64 * vs;
+        bool ok = true;
+
+        auto write_o = [&](int j) -> bool {  // read O_j out of TMEM, normalise, store
+            if (!wwait(&m->o_full[j & 1], (uint32_t)((j >> 1) & 1))) return false;
+            tc_fence_after();
+            uint32_t a[32], c[32];
+            const uint32_t tO = tmem + C::TM_O + 64 * (j & 1) + lane_base;
+            tmem_ld32(tO, a);
+            tmem_ld32(tO + 32, c);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&m->o_free[j & 1]);
+            float scale = 1.0f;
+            if (p.rmsnorm) {
+                float ss = 0.f;
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const float x = __uint_as_float(a[t]), y = __uint_as_float(c[t]);
+                    ss = fmaf(x, x, ss);
+                    ss = fmaf(y, y, ss);
+                }
+                if constexpr (C::NVS > 1) {
+                    if (r_ok) st_remote_f32(&m->ss_in[j & 1][r], partner, ss);
+                    mbar_arrive_remote(&m->ss_full[j & 1], partner);
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait<true>(&m->ss_full[j & 1], (uint32_t)((j >> 1) & 1),
+                                                    abort_flag, tlimit)))
+                        return false;
+                    if (r_ok) ss = ss + m->ss_in[j & 1][r];
+                }
+                scale = rsqrtf(ss * (1.0f / D) + 1e-6f);
+            }
+            const int nv = min(BETA, seq_len - j * BETA);
+            if (r_ok && r < nv) {
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    p.o + ((size_t)(seq_start + j * BETA + r) * p.H) * D + o_col);
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    dst[t] = make_uint4(
+                        pack_bf16x2(__uint_as_float(a[8 * t + 0]) * scale, __uint_as_float(a[8 * t + 1]) * scale),
+                        pack_bf16x2(__uint_as_float(a[8 * t + 2]) * scale, __uint_as_float(a[8 * t + 3]) * scale),
+                        pack_bf16x2(__uint_as_float(a[8 * t + 4]) * scale, __uint_as_float(a[8 * t + 5]) * scale),
+                        pack_bf16x2(__uint_as_float(a[8 * t + 6]) * scale, __uint_as_float(a[8 * t + 7]) * scale));
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    dst[4 + t] = make_uint4(
+                        pack_bf16x2(__uint_as_float(c[8 * t + 0]) * scale, __uint_as_float(c[8 * t + 1]) * scale),
+                        pack_bf16x2(__uint_as_float(c[8 * t + 2]) * scale, __uint_as_float(c[8 * t + 3]) * scale),
+                        pack_bf16x2(__uint_as_float(c[8 * t + 4]) * scale, __uint_as_float(c[8 * t + 5]) * scale),
+                        pack_bf16x2(__uint_as_float(c[8 * t + 6]) * scale, __uint_as_float(c[8 * t + 7]) * scale));
+            }
+            return true;
+        };
+
+        for (int b = 0; ok && b < nb; ++b) {
+            // (1) S_b -> P_b = bf16(S_b masked to j <= i), into the swizzled K-major tile
+            if (!wwait(&m->s_full[b & 1], (uint32_t)((b >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            if (b >= 1 && !wwait(&m->p_free, (uint32_t)((b - 1) & 1))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tS = tmem + C::TM_S + BETA * (b & 1) + lane_base;
+#pragma unroll 1
+            for (int cc = 0; cc < BETA / 32; ++cc) {
+                uint32_t s[32];
+                tmem_ld32(tS + 32 * cc, s);
+                tmem_ld_wait();
+                if (r_ok) {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int c0 = 32 * cc + 8 * t + 2 * u;
+                            const float x0 = c0 <= r ? __uint_as_float(s[8 * t + 2 * u]) : 0.f;
+                            const float x1 = c0 + 1 <= r ? __uint_as_float(s[8 * t + 2 * u + 1]) : 0.f;
+                            w[u] = pack_bf16x2(x0, x1);
+                        }
+                        const int col = 32 * cc + 8 * t;
+                        const uint32_t chunk = (uint32_t)(((col & 63) >> 3) ^ (r & 7));
+                        st_shared_v4(sP + (col >> 6) * C::BOX + r * 128 + (chunk << 4), w[0], w[1],
+                                     w[2], w[3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->p_ready);
+
+            // (2) snapshot of KV_{<b} (bf16, MN-major) for O_b += Q_b KV
+            if (b >= 1) {
+                if (!wwait(&m->kv_full, (uint32_t)((b - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t a[32], c[32];
+                const uint32_t tK = tmem + C::TM_KV + lane_base;
+                tmem_ld32(tK, a);
+                tmem_ld32(tK + 32, c);
+                tmem_ld_wait();
+                if (i_ok) {
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const uint32_t *src = t < 4 ? &a[8 * t] : &c[8 * (t - 4)];
+                        const uint32_t chunk = (uint32_t)(t ^ (i & 7));
+                        st_shared_v4(sSnap + i * 128 + (chunk << 4),
+                                     pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                                     pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                                     pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                                     pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&m->snap_ready);
+            }
+
+            // (3) the previous block's output
+            if (b >= 1 && !write_o(b - 1)) {
+                ok = false;
+                break;
+            }
+        }
+        if (ok && nb > 0) {
+            // final state K^T V of this sequence (fp32) and the last block's output
+            if (!wwait(&m->kv_full, (uint32_t)((nb - 1) & 1))) {
+                ok = false;
+            } else {
+                tc_fence_after();
+                uint32_t a[32], c[32];
+                const uint32_t tK = tmem + C::TM_KV + lane_base;
+                tmem_ld32(tK, a);
+                tmem_ld32(tK + 32, c);
+                tmem_ld_wait();
+                if (p.state != nullptr && i_ok) {
+                    float4 *dst = reinterpret_cast<float4 *>(
+                        p.state + (((size_t)sid * p.H + h) * D + i) * D + 64 * vs);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        dst[t] = make_float4(__uint_as_float(a[4 * t]), __uint_as_float(a[4 * t + 1]),
+                                             __uint_as_float(a[4 * t + 2]), __uint_as_float(a[4 * t + 3]));
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        dst[8 + t] = make_float4(__uint_as_float(c[4 * t]), __uint_as_float(c[4 * t + 1]),
+                                                 __uint_as_float(c[4 * t + 2]), __uint_as_float(c[4 * t + 3]));
+                }
+                ok = write_o(nb - 1);
+            }
+        } else if (nb == 0 && p.state != nullptr && i_ok) {
+            float4 *dst = reinterpret_cast<float4 *>(p.state + (((size_t)sid * p.H + h) * D + i) * D +
+                                                     64 * vs);
+            for (int t = 0; t < 16; ++t) dst[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (!ok) fail();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (C::NVS > 1) cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace la

@@ -1,0 +1,111 @@
+"""The C-ABI library loads, exports what the header declares, and rejects bad
+arguments on the host before any launch (CPU only: no compute call is made)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from long_context_04_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return api.lib()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(la_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for must in ("la_prefill", "la_decode_step", "la_state_out", "la_status_string",
+                 "la_get_device_status"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, text in [(0, "LA_OK"), (1, "LA_ERR_INVALID_ARG"), (2, "LA_ERR_UNSUPPORTED"),
+                       (3, "LA_ERR_CUDA"), (4, "LA_ERR_DEVICE_TIMEOUT"),
+                       (5, "LA_ERR_DEVICE_RANGE")]:
+        assert api.status_string(code) == text
+    assert api.status_string(99) == "LA_ERR_UNKNOWN"
+    assert L.la_version() >= 100
+
+
+FAKE = 0x10000  # an aligned, never-dereferenced address: validation fails before any use
+
+
+def _prefill(L, *, q=FAKE, o=FAKE, B=1, H=2, N=8, D=128, beta=128, cu=None, S=0, flags=1,
+             st=None):
+    cu_arr = None
+    if cu is not None:
+        arr = np.ascontiguousarray(np.asarray(cu, np.int32))
+        cu_arr = arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        _prefill.keep = arr
+    return L.la_prefill(q, FAKE, FAKE, o, B, H, N, D, beta, cu_arr, S, flags, st, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), api.LA_ERR_INVALID_ARG),
+    (dict(o=None), api.LA_ERR_INVALID_ARG),
+    (dict(q=FAKE + 2), api.LA_ERR_INVALID_ARG),          # misaligned
+    (dict(H=0), api.LA_ERR_INVALID_ARG),
+    (dict(N=-1), api.LA_ERR_INVALID_ARG),
+    (dict(B=0), api.LA_ERR_INVALID_ARG),
+    (dict(D=96), api.LA_ERR_UNSUPPORTED),
+    (dict(D=256), api.LA_ERR_UNSUPPORTED),
+    (dict(beta=32), api.LA_ERR_UNSUPPORTED),
+    (dict(beta=256), api.LA_ERR_UNSUPPORTED),
+    (dict(flags=1 | 64), api.LA_ERR_INVALID_ARG),        # unknown flag bit
+    (dict(flags=1 | 4, st=None), api.LA_ERR_INVALID_ARG),  # state requested, no buffer
+    (dict(cu=[0, 3, 8], S=2, B=2), api.LA_ERR_INVALID_ARG),  # cu_seqlens needs B == 1
+    (dict(cu=[1, 3, 8], S=2), api.LA_ERR_INVALID_ARG),   # must start at 0
+    (dict(cu=[0, 3, 7], S=2), api.LA_ERR_INVALID_ARG),   # must end at N
+    (dict(cu=[0, 5, 3, 8], S=3), api.LA_ERR_INVALID_ARG),  # decreasing
+    (dict(cu=[0], S=0), api.LA_ERR_INVALID_ARG),          # no sequence
+    (dict(cu=list(range(1026)), S=1025, N=1025), api.LA_ERR_UNSUPPORTED),  # too many
+])
+def test_prefill_rejects(L, kw, code):
+    assert _prefill(L, **kw) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, FAKE, FAKE, FAKE, FAKE, 2, 2, 128, 1), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, None, FAKE, 2, 2, 128, 1), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE + 4, FAKE, 2, 2, 128, 1), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 128, 1), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 2, 0, 128, 1), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 2, 2, 32, 1), api.LA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 2, 2, 128, 1 | 4), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 128, 1), api.LA_OK),   # empty batch: no-op
+])
+def test_decode_rejects(L, args, code):
+    assert L.la_decode_step(*args, None) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, FAKE, 2, 2, 128, None, 2), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, 3, 2, 128, None, 2), api.LA_ERR_INVALID_ARG),   # identity map overflows
+    ((FAKE, FAKE, 2, 2, 100, None, 2), api.LA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE + 8, 2, 2, 128, None, 2), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, 0, 2, 128, None, 2), api.LA_OK),                 # nothing to copy
+])
+def test_state_out_rejects(L, args, code):
+    assert L.la_state_out(*args, None) == code
