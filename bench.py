@@ -1,0 +1,501 @@
+"""Benchmark of the lightning-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_n131k|prefill_n16k] [--no-extras]
+
+A step is one la_prefill call over the long-context workload (B=1, H=64,
+N=131072, D=128, beta=128, bf16 inputs, fp32 accumulation, no output norm),
+with Q/K/V/O (8.6 GB) resident in HBM.  The inputs are far larger than the
+126 MB L2, so no flush is needed between steps.  ``value`` is prefill
+tokens/s over all ranks; the JSON line also carries the tensor-core view
+(TFLOP/s, % of bf16 peak), the decode step (B=256, H=64, D=128, fp32 state of a
+seeded N=4096 prefill; tokens/s and % of HBM bandwidth), the roofline of the
+prefill kernel, the end-to-end number through the C ABI with host buffers, and
+the fp64 oracle timed on the host cores as a CPU baseline.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload on its own
+GPU (independent problems, no data-path collective: weak scaling); the timed
+region is bracketed by barriers and the slowest rank's time is reported.
+
+``--impl reference`` times the fp64 CPU oracle on the same metric and unit,
+each step a bounded sample of the workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s (% HBM BW)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    # name: (B, N, H, D, beta)
+    "prefill_n131k": (1, 131072, 64, 128, 128),
+    "prefill_n16k": (1, 16384, 64, 128, 128),
+}
+DECODE = dict(B=256, H=64, D=128, N=4096, steps=64, chunk=32)
+KERNEL_SOURCES = [os.path.join(ROOT, "long_context_04_b200", "csrc", f)
+                  for f in ("prefill_tc.cuh", "la_device.cuh")]
+
+
+# ----------------------------------------------------------------------------- helpers
+def tiled_flops_per_token_head(D: int, beta: int) -> int:
+    """Tiled-form flops per token and head: 2*beta*D (QK^T) + 2*beta*D (PV) + 2*D*D (Q.KV)
+    + 2*D*D (K^T V), with beta x beta score blocks counted in full."""
+    return 4 * beta * D + 4 * D * D
+
+
+def useful_flops_per_token_head(D: int, beta: int) -> float:
+    """Causally useful flops: on average (beta+1)/2 keys per query inside a block."""
+    return 2 * D * (beta + 1) + 4 * D * D
+
+
+def prefill_bytes(T: int, H: int, D: int) -> int:
+    """Algorithmic HBM bytes of one prefill: read Q, K, V and write O, bf16."""
+    return 8 * T * H * D
+
+
+def decode_bytes(B: int, H: int, D: int) -> int:
+    """Per step: fp32 state read + write (8 D^2) and bf16 q, k, v, o (8 D) per (b, h)."""
+    return B * H * (8 * D * D + 8 * D)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_digest(paths) -> str:
+    """sha256 over the kernel's source files (the record is void once any of them changes)."""
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_record(kernel_srcs):
+    """DRAM bytes per token-head from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", "prefill_tc_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("source_sha256") == kernel_digest(kernel_srcs):
+            return rec
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks rather than guess
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    _NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+              0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+              0x100: "display_clock_setting"}
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self._NAMES.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_init():
+    """(rank, world, local_rank) from the torchrun environment; single process otherwise."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_setup(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_max(x: float, world: int, device=None) -> float:
+    """Maximum of a float over all ranks (every rank calls this in the same order)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(D: int, heads: int, tokens: int, seed: int = 0):
+    """A bounded sample of the workload for the fp64 oracle: `heads` heads x `tokens` tokens
+    (the first tokens of the sequence), drawn with the same recipe as the GPU inputs."""
+    import torch
+
+    from long_context_04_b200 import synth
+    q, k, v = synth.qkv(tokens, heads, D, seed=seed, dtype=torch.bfloat16, device="cpu")
+    return q, k, v
+
+
+def time_oracle_prefill(q, k, v, nthreads: int) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, want_o=True, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(B, N, H, D, beta, budget_s=12.0):
+    """fp64 oracle (recurrent form, the cheapest exact form) on the host cores.
+
+    Calibrates on a small sample, then times `cores` heads x L tokens sized for about
+    `budget_s` of wall time.  The value is in the metric's unit: tokens of the H-head
+    layer per second = (sampled tokens x sampled heads / H) / time."""
+    cores = max(1, os.cpu_count() or 1)
+    heads = min(H, cores)
+    q, k, v = oracle_sample(D, heads, 1024)
+    t = time_oracle_prefill(q, k, v, heads)
+    per_token = max(t / 1024.0, 1e-7)
+    L = int(max(1024, min(N, budget_s / per_token)))
+    L = (L // 1024) * 1024
+    q, k, v = oracle_sample(D, heads, L, seed=1)
+    t = time_oracle_prefill(q, k, v, heads)
+    value = L * heads / H / t
+    return {"value": value, "unit": "tokens/s", "cores": heads, "kind": "oracle",
+            "sample": f"fp64 recurrent form, {heads} heads x {L} tokens of the N={N} "
+                      f"sequence ({heads}/{H} of the heads), {t:.1f} s on {heads} threads; "
+                      f"value = sampled token-heads / {H} / time",
+            "seconds": t}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_init()
+    if rank != 0:
+        return 0
+    B, N, H, D, beta = WORKLOADS[args.workload]
+    cores = max(1, os.cpu_count() or 1)
+    heads = min(H, cores)
+    q, k, v = oracle_sample(D, heads, 1024)
+    per_token = max(time_oracle_prefill(q, k, v, heads) / 1024.0, 1e-7)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    L = int(max(256, min(N, budget / per_token)))
+    q, k, v = oracle_sample(D, heads, L, seed=1)
+    for _ in range(args.warmup):
+        time_oracle_prefill(q, k, v, heads)
+    times = [time_oracle_prefill(q, k, v, heads) for _ in range(args.steps)]
+    total = sum(times)
+    value = args.steps * L * heads / H / total
+    sample = (f"per step: fp64 recurrent oracle on {heads} heads x {L} tokens of the {args.workload} "
+              f"workload, {heads} threads; value = sampled token-heads / {H} / time")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(args.workload), "global_batch": B, "seq_len": N,
+                   "heads": H, "head_dim": D, "beta": beta, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": heads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_name(w: str) -> str:
+    B, N, H, D, beta = WORKLOADS[w]
+    return (f"lightning-attention causal prefill, B={B}, N={N}, H={H}, D={D}, beta={beta}, "
+            f"bf16 in / fp32 accumulate, no output norm")
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+
+    from long_context_04_b200 import api, build as lib_build, synth
+
+    rank, world, local = dist_init()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist_setup(world, "nccl")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lib_build.build()
+    api.lib()
+
+    B, N, H, D, beta = WORKLOADS[args.workload]
+    T = B * N
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+
+    with torch.cuda.stream(stream):
+        q, k, v = synth.qkv(T, H, D, seed=rank, dtype=torch.bfloat16, device=dev)
+        q, k, v = (x.view(B, N, H, D) for x in (q, k, v))
+        o = torch.empty_like(q)
+    stream.synchronize()
+
+    def step():
+        api.prefill(q, k, v, beta=beta, out=o, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    status = api.device_status(stream)
+    if status != api.LA_OK:
+        raise RuntimeError(f"device status after warm-up: {api.status_string(status)}")
+
+    # ---- timed region: K prefill launches, per-launch events on the launching stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_begin.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    dist_barrier(world)
+    local_ms = t_begin.elapsed_time(t_end)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = dist_max(local_ms, world, dev)
+    status = api.device_status(stream)
+    if status != api.LA_OK:
+        raise RuntimeError(f"device status after timing: {api.status_string(status)}")
+
+    tokens_total = T * world * args.steps
+    value = tokens_total / (ms / 1e3)
+    ms_per_step = ms / args.steps
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+    flops = tiled_flops_per_token_head(D, beta) * T * H
+    useful = useful_flops_per_token_head(D, beta) * T * H
+    alg_bytes = prefill_bytes(T, H, D)
+    tflops = flops / avg_launch_s / 1e12
+    hbm_gbs = alg_bytes / avg_launch_s / 1e9
+    peak_bw = float(peaks["hbm_gbs"])
+    peak_tf = float(peaks["bf16_tflops"])
+    trec = traffic_record(KERNEL_SOURCES)
+    traffic = None
+    if trec is not None:
+        traffic = float(trec["bytes_per_launch_per_token_head"]) * T * H
+    roofline = {"bound": "hbm", "achieved": hbm_gbs, "peak": peak_bw, "unit": "GB/s",
+                "frac": hbm_gbs / peak_bw, "traffic": traffic,
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "kernel": f"la::prefill_tc_kernel<{beta},{D}>"}
+    prefill_view = {"tflops_tiled": tflops, "pct_bf16_peak": 100.0 * tflops / peak_tf,
+                    "tflops_causal_useful": useful / avg_launch_s / 1e12,
+                    "bf16_peak_tflops": peak_tf,
+                    "roofline_ceiling_tflops": min(peak_tf, flops / alg_bytes * peak_bw / 1e3),
+                    "avg_launch_ms": avg_launch_s * 1e3,
+                    "flops_per_token_head": tiled_flops_per_token_head(D, beta)}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: Q, K, V iid N(0,1)/sqrt(D), seeded per rank",
+        "config": {"workload": workload_name(args.workload), "global_batch": B * world,
+                   "seq_len": N, "heads": H, "head_dim": D, "beta": beta,
+                   "parallelism": f"replicas x{world} (independent problems, no collective)",
+                   "l2": "inputs (8.6 GB) larger than the 126 MB L2; no flush"},
+        "prefill": prefill_view, "roofline": roofline, "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_extras:
+        line["e2e"] = e2e_prefill(args, api, torch, q, k, v, B, N, H, D, beta, world, dev)
+        line["decode"] = bench_decode(api, synth, torch, dev, stream, peak_bw, rank, world)
+    if rank == 0 and not args.no_extras:
+        line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def e2e_prefill(args, api, torch, q, k, v, B, N, H, D, beta, world, dev):
+    """Same metric through the C ABI with host buffers: each step copies Q, K, V from pinned
+    host memory, runs la_prefill and copies O back to pinned host memory."""
+    steps = 3
+    hq, hk, hv = (x.to("cpu").pin_memory() for x in (q, k, v))
+    ho = torch.empty_like(hq).pin_memory()
+    s = torch.cuda.Stream(device=dev)
+    dq, dk, dv, do = (torch.empty_like(q) for _ in range(4))
+
+    def one():
+        with torch.cuda.stream(s):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            api.prefill(dq, dk, dv, beta=beta, out=do, stream=s)
+            ho.copy_(do, non_blocking=True)
+
+    one()
+    s.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    e0.record(s)
+    for _ in range(steps):
+        one()
+    e1.record(s)
+    s.synchronize()
+    dist_barrier(world)
+    ms = dist_max(e0.elapsed_time(e1), world, dev)
+    nbytes = q.numel() * q.element_size()
+    del dq, dk, dv, do
+    return {"value": B * N * world * steps / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "steps": steps,
+            "note": "pinned host Q/K/V -> device, la_prefill, device O -> pinned host; one stream"}
+
+
+def bench_decode(api, synth, torch, dev, pstream, peak_bw, rank, world):
+    """Decode step B=256, H=64, D=128 on its own stream; state from seeded N=4096 prefills
+    (8 chunks of 32 sequences, handed over with la_state_out)."""
+    B, H, D, N, steps, chunk = (DECODE[x] for x in ("B", "H", "D", "N", "steps", "chunk"))
+    state = torch.empty(B, H, D, D, device=dev)
+    with torch.cuda.stream(pstream):
+        for c in range(B // chunk):
+            q, k, v = synth.qkv(chunk * N, H, D, seed=100 + c + 1000 * rank, dtype=torch.bfloat16,
+                                device=dev)
+            q, k, v = (x.view(chunk, N, H, D) for x in (q, k, v))
+            _, ws = api.prefill(q, k, v, beta=128, return_state=True, stream=pstream)
+            slots = torch.arange(c * chunk, (c + 1) * chunk, dtype=torch.int32, device=dev)
+            api.state_out(ws, state, slots, stream=pstream)
+            del q, k, v, ws
+    pstream.synchronize()
+    dstream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(dstream):
+        toks = [synth.decode_tokens(B, H, D, step=t, seed=rank, device=dev) for t in range(steps)]
+        outs = [torch.empty(B, H, D, dtype=torch.bfloat16, device=dev) for _ in range(steps)]
+    dstream.synchronize()
+    for t in range(3):  # warm-up on a copy of the state
+        scratch = state.clone()
+        api.decode_step(*toks[t], scratch, out=outs[t], stream=dstream)
+    dstream.synchronize()
+    del scratch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    ev[0].record(dstream)
+    for t in range(steps):
+        api.decode_step(*toks[t], state, out=outs[t], stream=dstream)
+        ev[t + 1].record(dstream)
+    dstream.synchronize()
+    dist_barrier(world)
+    per = [ev[t].elapsed_time(ev[t + 1]) for t in range(steps)]
+    med_ms = statistics.median(per)
+    total_ms = dist_max(ev[0].elapsed_time(ev[steps]), world, dev)
+    gbs = decode_bytes(B, H, D) / (med_ms / 1e3) / 1e9
+    status = api.device_status(dstream)
+    return {"workload": f"decode step, B={B}, H={H}, D={D}, bf16 q/k/v/o, fp32 state from a "
+                        f"seeded N={N} prefill, {steps} consecutive steps",
+            "tokens_per_s": B * world * steps / (total_ms / 1e3),
+            "ms_per_step_median": med_ms, "gbs_median_step": gbs, "pct_hbm": 100.0 * gbs / peak_bw,
+            "bytes_per_step": decode_bytes(B, H, D), "gpu_launches": steps,
+            "status": api.status_string(status), "stream": "own stream (not the prefill stream)"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill_n131k")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the prefill only (no e2e, decode or CPU baseline)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -57,7 +57,7 @@ typedef enum {
 
 /* Flags (bitwise OR). */
 enum {
-    LA_FP32 = 0,         /* q, k, v, o are fp32; fp32 FFMA arithmetic throughout */
+    LA_FP32 = 0,         /* q, k, v, o are fp32; CUDA-core arithmetic, fp64 accumulation */
     LA_BF16 = 1,         /* q, k, v, o are bf16; tensor-core bf16 products, fp32 accumulate */
     LA_OUT_RMSNORM = 2,  /* per-token, per-head RMSNorm over D of the output (eps 1e-6, unit weight) */
     LA_WRITE_STATE = 4   /* la_prefill writes each sequence's final KV state to state_ws */

@@ -3,7 +3,11 @@
 // Same block algorithm as the bf16 path (MiniMax-01, CSDN digest section 2.1;
 // mizuki blog appendix "key concepts"): per block b of BETA tokens,
 //     O_b = [(Q_b K_b^T) (.) M] V_b + Q_b KV,     KV += K_b^T V_b,
-// every product in fp32 (TF32 would not meet a 1e-5 relative error).
+// on the CUDA cores (TF32 tensor cores would not meet a 1e-5 relative error).
+// Inputs, outputs, scores and the state are stored in fp32; every dot product
+// is accumulated in fp64 registers (an fp32 x fp32 product is exact in fp64),
+// so a row whose sum cancels -- a one-token sequence with q.k near zero, say --
+// still comes out within a few fp32 roundings.
 // One CTA (256 threads) owns one (sequence, head); K_b, V_b and the D x D
 // state stay in shared memory, query rows are processed 16 at a time.
 #pragma once
@@ -62,23 +66,26 @@ __global__ void __launch_bounds__(256)
             // S = Q_tile K_b^T with the causal mask (key c <= query row)
             for (int x = tid; x < C::RT * BETA; x += C::THREADS) {
                 const int rr = x / BETA, c = x % BETA;
-                float acc = 0.f;
+                double acc = 0.0;
                 if (c <= r0 + rr) {
 #pragma unroll 8
-                    for (int d = 0; d < D; ++d) acc = fmaf(sQ[rr * D + d], sK[c * D + d], acc);
+                    for (int d = 0; d < D; ++d)
+                        acc = fma((double)sQ[rr * D + d], (double)sK[c * D + d], acc);
                 }
-                sS[x] = acc;
+                sS[x] = (float)acc;
             }
             __syncthreads();
             // O = S V_b + Q_tile KV
             for (int x = tid; x < C::RT * D; x += C::THREADS) {
                 const int rr = x / D, j = x % D;
-                float intra = 0.f, inter = 0.f;
+                double intra = 0.0, inter = 0.0;
                 const int cmax = min(r0 + rr, BETA - 1);
-                for (int c = 0; c <= cmax; ++c) intra = fmaf(sS[rr * BETA + c], sV[c * D + j], intra);
+                for (int c = 0; c <= cmax; ++c)
+                    intra = fma((double)sS[rr * BETA + c], (double)sV[c * D + j], intra);
 #pragma unroll 8
-                for (int i = 0; i < D; ++i) inter = fmaf(sQ[rr * D + i], sKV[i * D + j], inter);
-                sO[x] = intra + inter;
+                for (int i = 0; i < D; ++i)
+                    inter = fma((double)sQ[rr * D + i], (double)sKV[i * D + j], inter);
+                sO[x] = (float)(intra + inter);
             }
             __syncthreads();
             // optional RMSNorm per row, then store: one warp per row
@@ -87,11 +94,12 @@ __global__ void __launch_bounds__(256)
                 if (r0 + rr >= nv) continue;
                 float scale = 1.f;
                 if (rmsnorm) {
-                    float ss = 0.f;
-                    for (int j = lane; j < D; j += 32) ss = fmaf(sO[rr * D + j], sO[rr * D + j], ss);
+                    double ss = 0.0;
+                    for (int j = lane; j < D; j += 32)
+                        ss = fma((double)sO[rr * D + j], (double)sO[rr * D + j], ss);
 #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                    scale = 1.0f / sqrtf(ss / (float)D + 1e-6f);
+                    scale = (float)(1.0 / sqrt(ss / (double)D + 1e-6));
                 }
                 float *dst = o + ((size_t)(start + p0 + r0 + rr) * H + h) * D;
                 for (int j = lane; j < D; j += 32) dst[j] = sO[rr * D + j] * scale;
@@ -101,9 +109,9 @@ __global__ void __launch_bounds__(256)
         // KV += K_b^T V_b
         for (int x = tid; x < D * D; x += C::THREADS) {
             const int i = x / D, j = x % D;
-            float acc = sKV[x];
-            for (int c = 0; c < nv; ++c) acc = fmaf(sK[c * D + i], sV[c * D + j], acc);
-            sKV[x] = acc;
+            double acc = (double)sKV[x];
+            for (int c = 0; c < nv; ++c) acc = fma((double)sK[c * D + i], (double)sV[c * D + j], acc);
+            sKV[x] = (float)acc;
         }
     }
     __syncthreads();

@@ -9,22 +9,29 @@
 //
 // One CTA owns one work unit (sequence, head, 64-column slice of V/O).  With
 // D = 128 the two slices of a (sequence, head) form a 2-CTA cluster: both
-// recompute S = Q_b K_b^T (the second reads Q/K from L2) and exchange per-row
-// sums of squares through distributed shared memory for the RMSNorm.  All
-// four block contractions run on the tensor cores with fp32 accumulators in
-// TMEM; the D x 64 fp32 state lives in TMEM for the whole sequence.
+// compute S = Q_b K_b^T (the second reads Q/K from L2) and they exchange
+// per-row sums of squares through distributed shared memory for the RMSNorm.
+// The four block contractions run on the tensor cores with fp32 accumulators
+// in TMEM.  The state update is split to keep the serial chain short: the MMA
+// writes each block's increment dKV_b = K_b^T V_b into one of two TMEM
+// buffers, and the epilogue keeps the running fp32 state KV in registers
+// (one state row per thread), adds dKV_b, and writes the bf16 snapshot that
+// the next block's Q_{b+1} KV product reads.  So the MMA never waits for a
+// TMEM read before the next state update, and the whole state stays on chip
+// for the entire sequence.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: Q_b, K_b (D columns) and V_b (64 columns) into a
 //               ring of NST shared-memory stages.
 //   warp 1      TMEM owner and MMA issuer (lane 0 issues; the warp zeroes the
 //               V rows past a sequence end before they enter K^T V).
-//   warps 2..5  epilogue: S -> masked bf16 P (shared memory), fp32 state ->
-//               bf16 snapshot for the next block's Q_b KV, O -> (RMSNorm) ->
-//               bf16 global store, final state -> fp32 global store.
-// Per block the MMA issue order is: S_{b+1} (look-ahead), O_b = P_b V_b,
-// O_b += Q_b snap(KV_{<b}), KV += K_b^T V_b; one commit then releases the
-// stage, P, the O buffer and the state to the other roles.
+//   warps 2..5  group P: S_b -> causal mask -> bf16 P_b, written back into
+//               the first BETA/2 columns of S_b's TMEM buffer, where the
+//               O_b = P_b V_b product reads it as its A operand.
+//   warps 6..9  group O: KV += dKV_b, bf16 snapshot of KV, O_b -> (RMSNorm) ->
+//               bf16 global store, final fp32 state -> global store.
+// MMA issue order per block b: O_b = P_b V_b, dKV_b = K_b^T V_b,
+// O_b += Q_b snap(KV_{<b}), release of the stage, then S_{b+1}.
 // Every wait is bounded (see mbar_wait); on a timeout the CTA records
 // DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -70,35 +77,42 @@ struct PrefillTcParams {
     SeqTable seqs;
 };
 
+#ifndef LA_PREFETCH_BLOCKS
+#define LA_PREFETCH_BLOCKS 0
+#endif
+
 template <int BETA, int D>
 struct TcCfg {
     static constexpr int NVS = D / 64;          // CTAs per (sequence, head)
-    static constexpr int DV = 64;               // output columns per CTA
     static constexpr int DB = D / 64;           // 64-column tiles in Q or K
     static constexpr int BOX = BETA * 128;      // one 64-column tile of BETA rows (bytes)
     static constexpr int STAGE = (2 * DB + 1) * BOX;
-    static constexpr int P_BYTES = (BETA / 64) * BOX;
-    static constexpr int SNAP_BYTES = D * 128;
+    static constexpr int SNAP_BYTES = D * 128;  // D rows x 64 bf16
     static constexpr int SMEM_LIMIT = 227 * 1024;
     static constexpr int MISC = 2048;
-    static constexpr int NST_FIT = (SMEM_LIMIT - 1024 - P_BYTES - SNAP_BYTES - MISC) / STAGE;
+    static constexpr int NST_FIT =
+        (SMEM_LIMIT - 1024 - 2 * SNAP_BYTES - MISC) / STAGE;
     static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
     static_assert(NST >= 2, "shared memory budget");
-    static constexpr int OFF_P = NST * STAGE;
-    static constexpr int OFF_SNAP = OFF_P + P_BYTES;
-    static constexpr int OFF_MISC = OFF_SNAP + SNAP_BYTES;
+    // Blocks ahead of the TMA ring whose tiles are prefetched into L2, so that a
+    // stage load is served from L2 rather than waiting on HBM.
+    static constexpr int PF = LA_PREFETCH_BLOCKS;
+    static constexpr int OFF_SNAP = NST * STAGE;              // two snapshot buffers
+    static constexpr int OFF_MISC = OFF_SNAP + 2 * SNAP_BYTES;
     // At least 120 KB so that no two CTAs share an SM: each allocates all 512
     // TMEM columns, and a second resident CTA would block in tcgen05.alloc.
     static constexpr int SMEM_USED = 1024 + OFF_MISC + MISC;
     static constexpr int SMEM_BYTES = SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
-    // TMEM columns
-    static constexpr int TM_S = 0;              // two BETA-column S buffers
-    static constexpr int TM_O = 2 * BETA;       // two 64-column O buffers
-    static constexpr int TM_KV = 2 * BETA + 128;
+    static_assert(SMEM_USED <= SMEM_LIMIT, "shared memory budget");
+    // TMEM columns: S[2] (BETA each; P overwrites the first BETA/2 of each),
+    // O[2] (64 each), dKV[2] (64 each)
+    static constexpr int TM_S = 0;
+    static constexpr int TM_O = 2 * BETA;
+    static constexpr int TM_DKV = 2 * BETA + 128;
     static constexpr int TMEM_COLS = 512;
-    static_assert(TM_KV + 64 <= TMEM_COLS, "TMEM budget");
-    static constexpr int EPI_THREADS = 128;
-    static constexpr int THREADS = 64 + EPI_THREADS;
+    static_assert(TM_DKV + 128 <= TMEM_COLS, "TMEM budget");
+    static constexpr int GROUP = 128;           // threads of one epilogue group
+    static constexpr int THREADS = 64 + 2 * GROUP;
     static constexpr uint32_t ID_S = idesc_bf16_f32(BETA, BETA, 0, 0);
     static constexpr uint32_t ID_PV = idesc_bf16_f32(BETA, 64, 0, 1);
     static constexpr uint32_t ID_QKV = idesc_bf16_f32(BETA, 64, 0, 1);
@@ -113,10 +127,10 @@ struct TcMisc {
     uint64_t s_full[2];
     uint64_t o_full[2];
     uint64_t o_free[2];
+    uint64_t dkv_full[2];
+    uint64_t dkv_free[2];
     uint64_t ss_full[2];
     uint64_t p_ready;
-    uint64_t p_free;
-    uint64_t kv_full;
     uint64_t snap_ready;
     uint64_t drain;
     uint32_t tmem_base;
@@ -158,13 +172,13 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&m->s_full[i], 1);
             mbar_init(&m->o_full[i], 1);
-            mbar_init(&m->o_free[i], C::EPI_THREADS);
-            mbar_init(&m->ss_full[i], C::EPI_THREADS);
+            mbar_init(&m->o_free[i], C::GROUP);
+            mbar_init(&m->dkv_full[i], 1);
+            mbar_init(&m->dkv_free[i], C::GROUP);
+            mbar_init(&m->ss_full[i], C::GROUP);
         }
-        mbar_init(&m->p_ready, C::EPI_THREADS);
-        mbar_init(&m->p_free, 1);
-        mbar_init(&m->kv_full, 1);
-        mbar_init(&m->snap_ready, C::EPI_THREADS);
+        mbar_init(&m->p_ready, C::GROUP);
+        mbar_init(&m->snap_ready, C::GROUP);
         mbar_init(&m->drain, 1);
         m->abort_flag = 0;
         fence_mbarrier_init_cluster();
@@ -198,7 +212,18 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         // ------------------------------------------------------------ producer
         int issued = 0;
         if (lane == 0) {
+            auto prefetch = [&](int j) {
+                const int row = seq_start + j * BETA;
+                for (int c = 0; c < C::DB; ++c) {
+                    tma_prefetch_l2_2d(&p.tmap_q, h * D + 64 * c, row);
+                    tma_prefetch_l2_2d(&p.tmap_k, h * D + 64 * c, row);
+                }
+                tma_prefetch_l2_2d(&p.tmap_v, h * D + 64 * vs, row);
+            };
+            if constexpr (C::PF > 0)
+                for (int j = C::NST; j < C::NST + C::PF && j < nb; ++j) prefetch(j);
             for (int b = 0; b < nb; ++b) {
+                if (C::PF > 0 && b + C::NST + C::PF < nb) prefetch(b + C::NST + C::PF);
                 const int st = b % C::NST;
                 const uint32_t ph = (uint32_t)((b / C::NST) & 1);
                 if (!mbar_wait(&m->empty[st], ph ^ 1u, abort_flag, tlimit)) {
@@ -224,10 +249,6 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         bool any_issued = false;
-        const uint32_t tS[2] = {tmem + C::TM_S, tmem + C::TM_S + BETA};
-        const uint32_t tO[2] = {tmem + C::TM_O, tmem + C::TM_O + 64};
-        const uint32_t tKV = tmem + C::TM_KV;
-        const uint32_t sP = sbase + C::OFF_P, sSnap = sbase + C::OFF_SNAP;
 
         // Wait for block j's tiles, zero the V rows past the sequence end, issue S_j.
         auto stage_in = [&](int j) -> bool {
@@ -244,11 +265,12 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t sa = stage_addr(st);
+                const uint32_t dS = tmem + C::TM_S + BETA * (j & 1);
+                const uint64_t qd = desc_kmajor_sw128(sa), kd = desc_kmajor_sw128(sa + C::DB * C::BOX);
+#pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off = (uint32_t)((ks >> 2) * C::BOX + (ks & 3) * 32);
-                    mma_bf16_ss(tS[j & 1], desc_kmajor_sw128(sa + off),
-                                desc_kmajor_sw128(sa + C::DB * C::BOX + off), C::ID_S,
-                                ks > 0 ? 1u : 0u);
+                    mma_bf16_ss(dS, desc_add(qd, off), desc_add(kd, off), C::ID_S, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(&m->s_full[j & 1]);
             }
@@ -257,30 +279,40 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             return true;
         };
 
+        // Per block b: O_b = P_b V_b, dKV_b = K_b^T V_b, O_b += Q_b snap(KV_{<b}); the stage
+        // is released; then S_{b+1} = Q_{b+1} K_{b+1}^T.  S_{b+1} is issued last so that its
+        // tiles, loaded when stage b-1 was released, have had a whole block to arrive; the
+        // epilogue turns S_{b+1} into P_{b+1} while the tensor pipe drains block b.
         bool ok = nb == 0 || stage_in(0);
         for (int b = 0; ok && b < nb; ++b) {
-            if (b + 1 < nb && !stage_in(b + 1)) {
-                ok = false;
-                break;
-            }
             const int st = b % C::NST;
             const uint32_t sa = stage_addr(st);
             const uint32_t sV = sa + 2 * C::DB * C::BOX;
+            const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
+            const uint32_t dKV = tmem + C::TM_DKV + 64 * (b & 1);
             if (!wwait(&m->p_ready, (uint32_t)(b & 1))) {
                 ok = false;
                 break;
             }
-            if (b >= 2 && !wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1))) {
+            if (b >= 2 && (!wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)) ||
+                           !wwait(&m->dkv_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            if (lane == 0) {  // O_b = P_b V_b
+            if (lane == 0) {
+                // O_b = P_b V_b, P_b from TMEM: 16 keys = 8 packed columns per K-step
+                const uint32_t tP = tmem + C::TM_S + BETA * (b & 1);
+                const uint64_t vd = desc_mnmajor_sw128(sV, C::BOX);
+                const uint64_t ktd = desc_mnmajor_sw128(sa + C::DB * C::BOX, C::BOX);
+#pragma unroll
                 for (int ks = 0; ks < BETA / 16; ++ks)
-                    mma_bf16_ss(tO[b & 1],
-                                desc_kmajor_sw128(sP + (ks >> 2) * C::BOX + (ks & 3) * 32),
-                                desc_mnmajor_sw128(sV + ks * 2048, C::BOX), C::ID_PV,
+                    mma_bf16_ts(dO, tP + 8 * ks, desc_add(vd, ks * 2048), C::ID_PV, ks > 0 ? 1u : 0u);
+#pragma unroll
+                for (int ks = 0; ks < BETA / 16; ++ks)  // dKV_b = K_b^T V_b
+                    mma_bf16_ss(dKV, desc_add(ktd, ks * 2048), desc_add(vd, ks * 2048), C::ID_KV,
                                 ks > 0 ? 1u : 0u);
+                mma_commit(&m->dkv_full[b & 1]);
             }
             __syncwarp();
             if (b >= 1) {
@@ -290,24 +322,24 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {  // O_b += Q_b snap(KV_{<b})
+                    const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (b & 1);
+                    const uint64_t qd = desc_kmajor_sw128(sa), sd = desc_mnmajor_sw128(sSnap, C::BOX);
+#pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks)
-                        mma_bf16_ss(tO[b & 1],
-                                    desc_kmajor_sw128(sa + (ks >> 2) * C::BOX + (ks & 3) * 32),
-                                    desc_mnmajor_sw128(sSnap + ks * 2048, C::BOX), C::ID_QKV, 1u);
+                        mma_bf16_ss(dO, desc_add(qd, (uint32_t)((ks >> 2) * C::BOX + (ks & 3) * 32)),
+                                    desc_add(sd, ks * 2048), C::ID_QKV, 1u);
                 }
                 __syncwarp();
             }
-            if (lane == 0) {  // KV += K_b^T V_b
-                for (int ks = 0; ks < BETA / 16; ++ks)
-                    mma_bf16_ss(tKV, desc_mnmajor_sw128(sa + C::DB * C::BOX + ks * 2048, C::BOX),
-                                desc_mnmajor_sw128(sV + ks * 2048, C::BOX), C::ID_KV,
-                                (b > 0 || ks > 0) ? 1u : 0u);
+            if (lane == 0) {
                 mma_commit(&m->o_full[b & 1]);
-                mma_commit(&m->p_free);
-                mma_commit(&m->kv_full);
                 mma_commit(&m->empty[st]);
             }
             __syncwarp();
+            if (b + 1 < nb && !stage_in(b + 1)) {
+                ok = false;
+                break;
+            }
         }
         if (!ok) fail();
         if (any_issued && lane == 0) {  // every issued MMA has finished before TMEM is freed
@@ -315,16 +347,55 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             mbar_wait(&m->drain, 0u, nullptr, tlimit);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ epilogue
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ group P
+        // S_b and P_b share a TMEM buffer: chunk cc reads S columns [64cc, 64cc+64)
+        // and writes P columns [32cc, 32cc+32), which lie in S columns already read.
+        // S_{b+2} reuses the buffer only after O_b = P_b V_b, in MMA issue order.
         const int q = warp & 3;                    // TMEM lane quadrant of this warp
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int r = BETA == 128 ? 32 * q + lane : 16 * q + lane;   // row of the block
+        const int r = BETA == 128 ? 32 * q + lane : 16 * q + lane;   // query row in the block
+        bool ok = true;
+        for (int b = 0; b < nb; ++b) {
+            if (!wwait(&m->s_full[b & 1], (uint32_t)((b >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tS = tmem + C::TM_S + BETA * (b & 1) + lane_base;
+#pragma unroll 1
+            for (int cc = 0; cc < BETA / 64; ++cc) {
+                uint32_t s0[32], s1[32], w[32];
+                tmem_ld32(tS + 64 * cc, s0);
+                tmem_ld32(tS + 64 * cc + 32, s1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const uint32_t *s = u < 16 ? &s0[2 * u] : &s1[2 * (u - 16)];
+                    const int c0 = 64 * cc + 2 * u;
+                    const float x0 = c0 <= r ? __uint_as_float(s[0]) : 0.f;
+                    const float x1 = c0 + 1 <= r ? __uint_as_float(s[1]) : 0.f;
+                    w[u] = pack_bf16x2(x0, x1);
+                }
+                tmem_st32(tS + 32 * cc, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&m->p_ready);
+        }
+        if (!ok) fail();
+    } else {
+        // ------------------------------------------------------------ group O
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int r = BETA == 128 ? 32 * q + lane : 16 * q + lane;   // query row in the block
         const bool r_ok = BETA == 128 || lane < 16;
         const int i = D == 128 ? 32 * q + lane : 16 * q + lane;      // state row
         const bool i_ok = D == 128 || lane < 16;
-        const uint32_t sP = sbase + C::OFF_P, sSnap = sbase + C::OFF_SNAP;
         const size_t o_col = (size_t)h * D + 64 * vs;
+        float kv[64];                                              // KV[i][64 vs .. 64 vs + 63]
+#pragma unroll
+        for (int t = 0; t < 64; ++t) kv[t] = 0.f;
         bool ok = true;
 
         auto write_o = [&](int j) -> bool {  // read O_j out of TMEM, normalise, store
@@ -362,126 +433,70 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 uint4 *dst = reinterpret_cast<uint4 *>(
                     p.o + ((size_t)(seq_start + j * BETA + r) * p.H) * D + o_col);
 #pragma unroll
-                for (int t = 0; t < 4; ++t)
+                for (int t = 0; t < 8; ++t) {
+                    const uint32_t *src = t < 4 ? &a[8 * t] : &c[8 * (t - 4)];
                     dst[t] = make_uint4(
-                        pack_bf16x2(__uint_as_float(a[8 * t + 0]) * scale, __uint_as_float(a[8 * t + 1]) * scale),
-                        pack_bf16x2(__uint_as_float(a[8 * t + 2]) * scale, __uint_as_float(a[8 * t + 3]) * scale),
-                        pack_bf16x2(__uint_as_float(a[8 * t + 4]) * scale, __uint_as_float(a[8 * t + 5]) * scale),
-                        pack_bf16x2(__uint_as_float(a[8 * t + 6]) * scale, __uint_as_float(a[8 * t + 7]) * scale));
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    dst[4 + t] = make_uint4(
-                        pack_bf16x2(__uint_as_float(c[8 * t + 0]) * scale, __uint_as_float(c[8 * t + 1]) * scale),
-                        pack_bf16x2(__uint_as_float(c[8 * t + 2]) * scale, __uint_as_float(c[8 * t + 3]) * scale),
-                        pack_bf16x2(__uint_as_float(c[8 * t + 4]) * scale, __uint_as_float(c[8 * t + 5]) * scale),
-                        pack_bf16x2(__uint_as_float(c[8 * t + 6]) * scale, __uint_as_float(c[8 * t + 7]) * scale));
+                        pack_bf16x2(__uint_as_float(src[0]) * scale, __uint_as_float(src[1]) * scale),
+                        pack_bf16x2(__uint_as_float(src[2]) * scale, __uint_as_float(src[3]) * scale),
+                        pack_bf16x2(__uint_as_float(src[4]) * scale, __uint_as_float(src[5]) * scale),
+                        pack_bf16x2(__uint_as_float(src[6]) * scale, __uint_as_float(src[7]) * scale));
+                }
             }
             return true;
         };
 
-        for (int b = 0; ok && b < nb; ++b) {
-            // (1) S_b -> P_b = bf16(S_b masked to j <= i), into the swizzled K-major tile
-            if (!wwait(&m->s_full[b & 1], (uint32_t)((b >> 1) & 1))) {
-                ok = false;
-                break;
-            }
-            if (b >= 1 && !wwait(&m->p_free, (uint32_t)((b - 1) & 1))) {
+        for (int b = 0; b < nb; ++b) {
+            // (1) KV += dKV_b; the bf16 snapshot of KV_{<b+1} for O_{b+1} += Q_{b+1} KV
+            if (!wwait(&m->dkv_full[b & 1], (uint32_t)((b >> 1) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t tS = tmem + C::TM_S + BETA * (b & 1) + lane_base;
-#pragma unroll 1
-            for (int cc = 0; cc < BETA / 32; ++cc) {
-                uint32_t s[32];
-                tmem_ld32(tS + 32 * cc, s);
-                tmem_ld_wait();
-                if (r_ok) {
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int c0 = 32 * cc + 8 * t + 2 * u;
-                            const float x0 = c0 <= r ? __uint_as_float(s[8 * t + 2 * u]) : 0.f;
-                            const float x1 = c0 + 1 <= r ? __uint_as_float(s[8 * t + 2 * u + 1]) : 0.f;
-                            w[u] = pack_bf16x2(x0, x1);
-                        }
-                        const int col = 32 * cc + 8 * t;
-                        const uint32_t chunk = (uint32_t)(((col & 63) >> 3) ^ (r & 7));
-                        st_shared_v4(sP + (col >> 6) * C::BOX + r * 128 + (chunk << 4), w[0], w[1],
-                                     w[2], w[3]);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&m->p_ready);
-
-            // (2) snapshot of KV_{<b} (bf16, MN-major) for O_b += Q_b KV
-            if (b >= 1) {
-                if (!wwait(&m->kv_full, (uint32_t)((b - 1) & 1))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+            {
                 uint32_t a[32], c[32];
-                const uint32_t tK = tmem + C::TM_KV + lane_base;
+                const uint32_t tK = tmem + C::TM_DKV + 64 * (b & 1) + lane_base;
                 tmem_ld32(tK, a);
                 tmem_ld32(tK + 32, c);
                 tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&m->dkv_free[b & 1]);
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    kv[t] += __uint_as_float(a[t]);
+                    kv[32 + t] += __uint_as_float(c[t]);
+                }
+            }
+            if (b + 1 < nb) {
+                // Buffer (b+1)&1 was last read by O_{b-1} += Q_{b-1} KV, which finished
+                // before dKV_b (MMAs complete in issue order), so it is free here.
+                const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * ((b + 1) & 1);
                 if (i_ok) {
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
-                        const uint32_t *src = t < 4 ? &a[8 * t] : &c[8 * (t - 4)];
                         const uint32_t chunk = (uint32_t)(t ^ (i & 7));
                         st_shared_v4(sSnap + i * 128 + (chunk << 4),
-                                     pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                                     pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                                     pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
-                                     pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+                                     pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
+                                     pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
+                                     pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
+                                     pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
                     }
                 }
                 fence_proxy_async_smem();
-                tc_fence_before();
                 mbar_arrive(&m->snap_ready);
             }
-
-            // (3) the previous block's output
+            // (2) the previous block's output
             if (b >= 1 && !write_o(b - 1)) {
                 ok = false;
                 break;
             }
         }
-        if (ok && nb > 0) {
-            // final state K^T V of this sequence (fp32) and the last block's output
-            if (!wwait(&m->kv_full, (uint32_t)((nb - 1) & 1))) {
-                ok = false;
-            } else {
-                tc_fence_after();
-                uint32_t a[32], c[32];
-                const uint32_t tK = tmem + C::TM_KV + lane_base;
-                tmem_ld32(tK, a);
-                tmem_ld32(tK + 32, c);
-                tmem_ld_wait();
-                if (p.state != nullptr && i_ok) {
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        p.state + (((size_t)sid * p.H + h) * D + i) * D + 64 * vs);
-#pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        dst[t] = make_float4(__uint_as_float(a[4 * t]), __uint_as_float(a[4 * t + 1]),
-                                             __uint_as_float(a[4 * t + 2]), __uint_as_float(a[4 * t + 3]));
-#pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        dst[8 + t] = make_float4(__uint_as_float(c[4 * t]), __uint_as_float(c[4 * t + 1]),
-                                                 __uint_as_float(c[4 * t + 2]), __uint_as_float(c[4 * t + 3]));
-                }
-                ok = write_o(nb - 1);
-            }
-        } else if (nb == 0 && p.state != nullptr && i_ok) {
+        if (ok && nb > 0) ok = write_o(nb - 1);
+        if (ok && p.state != nullptr && i_ok) {  // final state K^T V of the sequence, fp32
             float4 *dst = reinterpret_cast<float4 *>(p.state + (((size_t)sid * p.H + h) * D + i) * D +
                                                      64 * vs);
-            for (int t = 0; t < 16; ++t) dst[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                dst[t] = make_float4(kv[4 * t], kv[4 * t + 1], kv[4 * t + 2], kv[4 * t + 3]);
         }
         if (!ok) fail();
     }
