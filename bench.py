@@ -480,18 +480,54 @@ def bench_decode(api, synth, torch, dev, pstream, peak_bw, rank, world):
             "status": api.status_string(status), "stream": "own stream (not the prefill stream)"}
 
 
+def run_decode_small(args):
+    """Decode-only run on one GPU (B=64, H=64, D=128), for profiling the decode kernel."""
+    import torch
+
+    from long_context_04_b200 import api, build as lib_build, synth
+    lib_build.build()
+    B, H, D = 64, 64, 128
+    dev = torch.device("cuda", 0)
+    g = synth.generator(7, dev)
+    state = torch.randn(B, H, D, D, generator=g, device=dev, dtype=torch.float32)
+    toks = [synth.decode_tokens(B, H, D, step=t, seed=0, device=dev)
+            for t in range(args.steps + args.warmup)]
+    out = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
+    for t in range(args.warmup):
+        api.decode_step(*toks[t], state, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(args.steps):
+        api.decode_step(*toks[args.warmup + t], state, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, _ = load_peaks()
+    gbs = decode_bytes(B, H, D) / (ms / 1e3) / 1e9
+    print(json.dumps({"workload": f"decode step B={B} H={H} D={D} (profiling case)",
+                      "ms_per_step": ms, "gbs": gbs, "pct_hbm": 100 * gbs / peaks["hbm_gbs"],
+                      "status": api.status_string(api.device_status())}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill_n131k")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode_b64"],
+                    default="prefill_n131k",
+                    help="decode_b64: decode steps only, B=64 H=64 D=128 with a seeded random "
+                         "fp32 state (256 MB, larger than L2); a small case for profiling")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the prefill only (no e2e, decode or CPU baseline)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload == "decode_b64":
+        return run_decode_small(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
