@@ -46,7 +46,8 @@ WORKLOADS = {
 }
 DECODE = dict(B=256, H=64, D=128, N=4096, steps=64, chunk=32)
 KERNEL_SOURCES = [os.path.join(ROOT, "long_context_04_b200", "csrc", f)
-                  for f in ("prefill_tc.cuh", "la_device.cuh")]
+                  for f in ("prefill_pair.cuh", "prefill_tc.cuh", "la_device.cuh")]
+PREFILL_KERNEL = "la::prefill_pair_kernel (beta=128, D=128)"
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -92,7 +93,7 @@ def kernel_digest(paths) -> str:
 
 def traffic_record(kernel_srcs):
     """DRAM bytes per token-head from the committed ncu summary, if it was taken on this source."""
-    path = os.path.join(ROOT, "profiles", "prefill_tc_traffic.json")
+    path = os.path.join(ROOT, "profiles", "prefill_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -363,7 +364,7 @@ def run_ours(args):
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_launch": alg_bytes,
-                "kernel": f"la::prefill_tc_kernel<{beta},{D}>"}
+                "kernel": PREFILL_KERNEL}
     prefill_view = {"tflops_tiled": tflops, "pct_bf16_peak": 100.0 * tflops / peak_tf,
                     "tflops_causal_useful": useful / avg_launch_s / 1e12,
                     "bf16_peak_tflops": peak_tf,

@@ -12,6 +12,7 @@
 
 #include "decode.cuh"
 #include "prefill_simt.cuh"
+#include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
 
 namespace {
@@ -73,6 +74,27 @@ la_status launch_tc(const PrefillTcParams &p, int units, cudaStream_t stream) {
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = C::NVS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status launch_pair(const la::PrefillPairParams &p, int pairs, cudaStream_t stream) {
+    using C = la::PairCfg;
+    auto kern = la::prefill_pair_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -164,9 +186,24 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
 
     if (flags & LA_BF16) {
         if (T == 0 && !want_state) return LA_OK;
+        const long long Tm = T > 0 ? T : 1;  // a tensor map needs a non-empty extent
+        if (beta == 128 && D == 128) {
+            // paired-CTA kernel: each CTA of a pair loads half of the rows / columns
+            la::PrefillPairParams pp;
+            std::memset(&pp, 0, sizeof pp);
+            if (!make_map(&pp.tmap_q64, q, Tm, H, D, 64) || !make_map(&pp.tmap_k64, k, Tm, H, D, 64) ||
+                !make_map(&pp.tmap_k128, k, Tm, H, D, 128) || !make_map(&pp.tmap_v128, v, Tm, H, D, 128))
+                return LA_ERR_CUDA;
+            pp.o = static_cast<__nv_bfloat16 *>(o);
+            pp.state = state;
+            pp.H = H;
+            pp.rmsnorm = rms;
+            pp.timeout_ns = kWaitLimitNs;
+            pp.seqs = seqs;
+            return launch_pair(pp, S * H, stream);
+        }
         PrefillTcParams p;
         std::memset(&p, 0, sizeof p);
-        const long long Tm = T > 0 ? T : 1;  // a tensor map needs a non-empty extent
         if (!make_map(&p.tmap_q, q, Tm, H, D, beta) || !make_map(&p.tmap_k, k, Tm, H, D, beta) ||
             !make_map(&p.tmap_v, v, Tm, H, D, beta))
             return LA_ERR_CUDA;
@@ -177,7 +214,6 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
         p.timeout_ns = kWaitLimitNs;
         p.seqs = seqs;
         const int units = S * H * (D / 64);
-        if (beta == 128 && D == 128) return launch_tc<128, 128>(p, units, stream);
         if (beta == 64 && D == 128) return launch_tc<64, 128>(p, units, stream);
         if (beta == 128 && D == 64) return launch_tc<128, 64>(p, units, stream);
         return launch_tc<64, 64>(p, units, stream);
