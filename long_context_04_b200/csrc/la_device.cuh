@@ -74,6 +74,18 @@ __device__ __forceinline__ void st_remote_f32(float *local_addr, uint32_t cta_ra
         : "memory");
 }
 
+// Non-blocking probe: true once the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -130,6 +142,17 @@ __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
 }
 
 // 2-D tiled bulk tensor load into this CTA's shared memory, completing on `bar`.
+// Load into this CTA's shared memory, completing the transaction bytes on a
+// barrier given by its shared::cluster address, which may lie in the partner
+// CTA of the pair (the .cta_group::2 form).
+__device__ __forceinline__ void tma_load_2d_pairbar(uint32_t smem_dst, const void *tmap, int x, int y,
+                                                    uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2 "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const void *tmap, int x, int y,
                                             uint64_t *bar) {
     asm volatile(
@@ -211,6 +234,16 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster_addr) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             bar_cluster_addr)
+        : "memory");
+}
+
+// One commit that arrives on the barrier at the same shared-memory offset in
+// both CTAs of the pair (CTA mask 0b11).
+__device__ __forceinline__ void mma_commit_pair_both(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((unsigned short)3)
         : "memory");
 }
 
