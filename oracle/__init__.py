@@ -46,7 +46,7 @@ def _lib(path: str | None = None):
         lib = ctypes.CDLL(path)
         dp = ctypes.POINTER(ctypes.c_double)
         lp = ctypes.POINTER(ctypes.c_int64)
-        lib.la_oracle_prefill.argtypes = [ctypes.c_int, dp, dp, dp, dp, dp, ctypes.c_int64,
+        lib.la_oracle_prefill.argtypes = [ctypes.c_int, dp, dp, dp, dp, dp, dp, ctypes.c_int64,
                                           ctypes.c_int, ctypes.c_int, lp, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
         lib.la_oracle_prefill.restype = ctypes.c_int
@@ -104,16 +104,21 @@ _FORMS = {"quadratic": 0, "recurrent": 1, "blocked": 2}
 
 def _prefill(form: str, q, k, v, cu_seqlens=None, *, beta: int = 0, rmsnorm: bool = False,
              eps: float = 1e-6, want_o: bool = True, want_state: bool = True,
-             nthreads: int | None = None):
+             initial_state=None, nthreads: int | None = None):
     q, k, v = _f64(q), _f64(k), _f64(v)
     if q.ndim != 3 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must share one [T, H, D] shape")
     T, H, D = q.shape
     cu = _cu(cu_seqlens, T)
     S = len(cu) - 1
+    x0 = None
+    if initial_state is not None:
+        x0 = _f64(initial_state)
+        if x0.shape != (S, H, D, D):
+            raise ValueError("initial_state must be [S, H, D, D]")
     o = np.zeros((T, H, D), np.float64) if want_o or form != "recurrent" else None
     st = np.zeros((S, H, D, D), np.float64) if want_state else None
-    rc = _lib(_ACTIVE[0]).la_oracle_prefill(_FORMS[form], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(st), T,
+    rc = _lib(_ACTIVE[0]).la_oracle_prefill(_FORMS[form], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(st), _ptr(x0), T,
                                   H, D, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), S,
                                   beta, int(rmsnorm), eps, nthreads or default_threads())
     if rc != 0:
@@ -121,21 +126,28 @@ def _prefill(form: str, q, k, v, cu_seqlens=None, *, beta: int = 0, rmsnorm: boo
     return o, st
 
 
-def quadratic(q, k, v, cu_seqlens=None, *, rmsnorm=False, eps=1e-6, nthreads=None):
-    """O = [(Q K^T) (.) M] V per sequence; returns (O, final state)."""
-    return _prefill("quadratic", q, k, v, cu_seqlens, rmsnorm=rmsnorm, eps=eps, nthreads=nthreads)
+def quadratic(q, k, v, cu_seqlens=None, *, rmsnorm=False, eps=1e-6, initial_state=None,
+              nthreads=None):
+    """O = q^T X + [(Q K^T) (.) M] V per sequence (X = initial_state, default 0);
+    returns (O, final state X + K^T V)."""
+    return _prefill("quadratic", q, k, v, cu_seqlens, rmsnorm=rmsnorm, eps=eps,
+                    initial_state=initial_state, nthreads=nthreads)
 
 
-def recurrent(q, k, v, cu_seqlens=None, *, rmsnorm=False, eps=1e-6, want_o=True, nthreads=None):
-    """Token-by-token state recurrence; returns (O or None, final state)."""
+def recurrent(q, k, v, cu_seqlens=None, *, rmsnorm=False, eps=1e-6, want_o=True,
+              initial_state=None, nthreads=None):
+    """Token-by-token state recurrence from KV = initial_state (default 0);
+    returns (O or None, final state)."""
     return _prefill("recurrent", q, k, v, cu_seqlens, rmsnorm=rmsnorm, eps=eps, want_o=want_o,
-                    nthreads=nthreads)
+                    initial_state=initial_state, nthreads=nthreads)
 
 
-def blocked(q, k, v, beta: int, cu_seqlens=None, *, rmsnorm=False, eps=1e-6, nthreads=None):
-    """Block-tiled lightning evaluation (intra left product + inter right product)."""
+def blocked(q, k, v, beta: int, cu_seqlens=None, *, rmsnorm=False, eps=1e-6, initial_state=None,
+            nthreads=None):
+    """Block-tiled lightning evaluation (intra left product + inter right product), the
+    state starting at initial_state (default 0)."""
     return _prefill("blocked", q, k, v, cu_seqlens, beta=beta, rmsnorm=rmsnorm, eps=eps,
-                    nthreads=nthreads)
+                    initial_state=initial_state, nthreads=nthreads)
 
 
 def decode_step(q, k, v, state, *, rmsnorm=False, eps=1e-6, nthreads=None):

@@ -26,6 +26,14 @@
  * requests get their own kernel): KV <- KV + k v^T, then o = q^T KV.  The
  * readout includes the current token, matching the causal diagonal j <= i.
  *
+ * Initial state (optional, state_in != NULL): a sequence may continue from a
+ * state X = KV at its start instead of 0, as a chunk of a longer sequence does
+ * (LASP+: local prefix sums of the chunk states, all-gathered, after which each
+ * chunk runs from the sum of the states before it -- mizuki blog, section 5
+ * "pretraining" and appendix "key concepts"; jvyan.cn article, section 3).  Then
+ *     O[i]  = q_i^T X + sum_{j <= i, j in s} (q_i . k_j) v_j,
+ *     KV_{start(s)-1} = X,   state = X + K_s^T V_s.
+ *
  * Layouts: q, k, v, o are [T][H][D] fp64 row-major (T = total tokens).
  * cu[] has S+1 non-decreasing entries from 0 to T; sequence s owns tokens
  * cu[s] .. cu[s+1]-1.  state is [S][H][D][D] with state[s][h][r][c] =
@@ -52,7 +60,8 @@ typedef struct {
     const double *q, *k, *v;
     double *o;      /* may be NULL (state only) */
     double *state;  /* may be NULL */
-    const double *state_in; /* decode: input state (may alias state) */
+    const double *state_in; /* decode: input state (may alias state); prefill: initial
+                               state per (sequence, head), or NULL for zero */
     int64_t T;
     int H, D, S;
     const int64_t *cu;
@@ -85,10 +94,18 @@ static void rmsnorm_row(double *x, int D, double eps) {
     for (int d = 0; d < D; ++d) x[d] = x[d] / r;
 }
 
+/* KV = X (an initial state), D x D row-major. */
+static void init_state(double *KV, const double *X, int D) {
+    for (int r = 0; r < D; ++r)
+        for (int c = 0; c < D; ++c)
+            KV[(size_t)r * D + c] = MUT(10) ? X[(size_t)c * D + r] : X[(size_t)r * D + c];
+}
+
 /* Quadratic masked form: O = [(Q K^T) (.) M] V, one row at a time. */
 static void run_quadratic(const job_t *J, int s, int h) {
     const int H = J->H, D = J->D;
     const int64_t a = J->cu[s], b = J->cu[s + 1];
+    const double *X = J->state_in ? J->state_in + ((size_t)s * H + h) * (size_t)D * D : NULL;
     for (int64_t i = a; i < b; ++i) {
         double *oi = rowm(J->o, i, h, H, D);
         for (int d = 0; d < D; ++d) oi[d] = 0.0;
@@ -98,11 +115,14 @@ static void run_quadratic(const job_t *J, int s, int h) {
             const double *vj = row(J->v, j, h, H, D);
             for (int d = 0; d < D; ++d) oi[d] += w * vj[d];
         }
+        if (X && !MUT(9))                                /* + q_i^T X */
+            for (int c = 0; c < D; ++c)
+                for (int r = 0; r < D; ++r) oi[c] += qi[r] * X[(size_t)r * D + c];
         if (J->rmsnorm) rmsnorm_row(oi, D, J->eps);
     }
     if (J->state) {
         double *st = J->state + ((size_t)s * H + h) * (size_t)D * D;
-        for (int r = 0; r < D * D; ++r) st[r] = 0.0;
+        for (int r = 0; r < D * D; ++r) st[r] = X && !MUT(11) ? X[r] : 0.0;
         for (int64_t j = a; j < b; ++j) {
             const double *kj = row(J->k, j, h, H, D), *vj = row(J->v, j, h, H, D);
             for (int r = 0; r < D; ++r)
@@ -116,6 +136,8 @@ static void run_recurrent(const job_t *J, int s, int h) {
     const int H = J->H, D = J->D;
     const int64_t a = J->cu[s], b = J->cu[s + 1];
     double *KV = (double *)calloc((size_t)D * D, sizeof(double));
+    if (J->state_in)                                     /* KV_{start-1} = X */
+        init_state(KV, J->state_in + ((size_t)s * H + h) * (size_t)D * D, D);
     for (int64_t i = a; i < b; ++i) {
         const double *ki = row(J->k, i, h, H, D), *vi = row(J->v, i, h, H, D);
         if (!MUT(5))
@@ -147,6 +169,8 @@ static void run_blocked(const job_t *J, int s, int h) {
     const int H = J->H, D = J->D, beta = J->beta;
     const int64_t a = J->cu[s], b = J->cu[s + 1];
     double *KV = (double *)calloc((size_t)D * D, sizeof(double));
+    if (J->state_in)                                     /* KV before the first block = X */
+        init_state(KV, J->state_in + ((size_t)s * H + h) * (size_t)D * D, D);
     double *intra = (double *)malloc((size_t)D * sizeof(double));
     double *inter = (double *)malloc((size_t)D * sizeof(double));
     for (int64_t p = a; p < b; p += beta) {
@@ -247,8 +271,8 @@ static int check_cu(const int64_t *cu, int S, int64_t T) {
 }
 
 int la_oracle_prefill(int form, const double *q, const double *k, const double *v, double *o,
-                      double *state, int64_t T, int H, int D, const int64_t *cu, int S,
-                      int beta, int rmsnorm, double eps, int nthreads) {
+                      double *state, const double *state_in, int64_t T, int H, int D,
+                      const int64_t *cu, int S, int beta, int rmsnorm, double eps, int nthreads) {
     if (H < 1 || D < 1 || T < 0 || form < 0 || form > 2) return -1;
     if (check_cu(cu, S, T)) return -2;
     if (form == 2 && beta < 1) return -3;
@@ -256,7 +280,7 @@ int la_oracle_prefill(int form, const double *q, const double *k, const double *
     if (!o && form != 1) return -4;
     job_t J;
     memset(&J, 0, sizeof J);
-    J.q = q; J.k = k; J.v = v; J.o = o; J.state = state;
+    J.q = q; J.k = k; J.v = v; J.o = o; J.state = state; J.state_in = state_in;
     J.T = T; J.H = H; J.D = D; J.S = S; J.cu = cu;
     J.rmsnorm = rmsnorm; J.eps = eps; J.beta = beta; J.form = form;
     return run_all(&J, nthreads);

@@ -10,7 +10,8 @@ or the mathematics fix:
   Q = K = e1 gives cumsum(V), orthogonal Q/K give zero, one token gives
   (q.k) v), the final state equal to a library K^T V;
 * invariants: linearity, scaling, packed = separate runs, block-size
-  independence, decode step = the next prefill row.
+  independence, decode step = the next prefill row, a sequence run in two
+  chunks (the second from the first one's state) = the single run.
 
 ``test_oracle.py`` runs them against the oracle; ``test_oracle_mutants.py``
 runs them against deliberately broken builds and requires each one to fail.
@@ -208,6 +209,74 @@ def pin_decode_is_next_row():
         o_dec, st_dec = oracle.decode_step(q[N:N + 1], k[N:N + 1], v[N:N + 1], st, rmsnorm=rms)
         _close(o_dec[0], o_full[N], 1e-11, "decode = next prefill row")
         _close(st_dec, st_full, 1e-11, "decode state")
+
+
+def _forms_with_state():
+    return {"quadratic": oracle.quadratic, "recurrent": oracle.recurrent,
+            "blocked3": lambda *a, **kw: oracle.blocked(a[0], a[1], a[2], 3, *a[3:], **kw),
+            "blocked16": lambda *a, **kw: oracle.blocked(a[0], a[1], a[2], 16, *a[3:], **kw)}
+
+
+def pin_chunked_equals_whole():
+    """Initial state: running each sequence in two chunks, the second one starting
+    from the first one's final state, reproduces the single run (rows and states)."""
+    T, H, D = 160, 2, 6
+    q, k, v = _rand((T, H, D), 40), _rand((T, H, D), 41), _rand((T, H, D), 42)
+    cu = [0, 45, 45, 160]                      # lengths 45, 0, 115
+    for rms in (False, True):
+        ref_o, ref_s = oracle.quadratic(q, k, v, cu, rmsnorm=rms)
+        for cut in ((0, 0, 0), (20, 0, 50), (45, 0, 115), (1, 0, 63)):
+            # chunk 1 of every sequence packed together, then chunk 2 of every sequence
+            c1, c2, rows1, rows2 = [0], [0], [], []
+            for s in range(3):
+                a, b = cu[s], cu[s + 1]
+                m = a + cut[s]
+                rows1 += list(range(a, m))
+                rows2 += list(range(m, b))
+                c1.append(len(rows1))
+                c2.append(len(rows2))
+            for name, fn in _forms_with_state().items():
+                o1, s1 = fn(q[rows1], k[rows1], v[rows1], c1, rmsnorm=rms)
+                o2, s2 = fn(q[rows2], k[rows2], v[rows2], c2, rmsnorm=rms, initial_state=s1)
+                _close(o1, ref_o[rows1], 1e-11, f"{name} chunk 1 cut {cut}")
+                _close(o2, ref_o[rows2], 1e-11, f"{name} chunk 2 cut {cut}")
+                _close(s2, ref_s, 1e-11, f"{name} state after chunk 2 cut {cut}")
+
+
+def pin_d1_cumsum_with_state():
+    """D = 1 with initial state x: O_i = q_i (x + sum_{j<=i} k_j v_j), a numpy cumsum."""
+    T = 40
+    q, k, v = _rand((T, 1, 1), 43), _rand((T, 1, 1), 44), _rand((T, 1, 1), 45)
+    x = np.array([[[[1.75]]]])
+    ref = q[:, 0, 0] * (1.75 + np.cumsum(k[:, 0, 0] * v[:, 0, 0]))
+    for name, fn in _forms_with_state().items():
+        o, st = fn(q, k, v, initial_state=x)
+        _close(o[:, 0, 0], ref, what=f"{name} D=1 cumsum with state")
+        _close(st[0, 0, 0, 0], ref[-1] / q[-1, 0, 0], 1e-11, f"{name} D=1 final state")
+
+
+def pin_one_token_with_state_is_decode():
+    """A one-token sequence continuing from state X is one decode step from X."""
+    H, D = 3, 7
+    q, k, v = _rand((1, H, D), 46), _rand((1, H, D), 47), _rand((1, H, D), 48)
+    X = _rand((1, H, D, D), 49)
+    for rms in (False, True):
+        o_dec, st_dec = oracle.decode_step(q, k, v, X, rmsnorm=rms)
+        for name, fn in _forms_with_state().items():
+            o, st = fn(q, k, v, rmsnorm=rms, initial_state=X)
+            _close(o, o_dec, 1e-11, f"{name} one token with state")
+            _close(st, st_dec, 1e-11, f"{name} state after one token")
+
+
+def pin_empty_sequence_keeps_state():
+    """A zero-length sequence leaves its initial state unchanged (exactly)."""
+    H, D = 2, 5
+    q = k = v = np.zeros((3, H, D))
+    X = _rand((2, H, D, D), 50)
+    for name, fn in _forms_with_state().items():
+        _, st = fn(q + _rand((3, H, D), 51), k + _rand((3, H, D), 52), v + _rand((3, H, D), 53),
+                   [0, 0, 3], initial_state=X)
+        assert np.array_equal(st[0], X[0]), f"{name} empty sequence state"
 
 
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

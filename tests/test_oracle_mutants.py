@@ -21,6 +21,9 @@ MUTANTS = {
     6: "decode readout before the state update",
     7: "intra-block mask not confined to the block (double count)",
     8: "RMSNorm over the sum instead of the mean of squares",
+    9: "initial state left out of the quadratic-form readout",
+    10: "initial state transposed in the recurrent and blocked forms",
+    11: "initial state left out of the quadratic-form final state",
 }
 
 
