@@ -60,7 +60,8 @@ enum {
     LA_FP32 = 0,         /* q, k, v, o are fp32; CUDA-core arithmetic, fp64 accumulation */
     LA_BF16 = 1,         /* q, k, v, o are bf16; tensor-core bf16 products, fp32 accumulate */
     LA_OUT_RMSNORM = 2,  /* per-token, per-head RMSNorm over D of the output (eps 1e-6, unit weight) */
-    LA_WRITE_STATE = 4   /* la_prefill writes each sequence's final KV state to state_ws */
+    LA_WRITE_STATE = 4,  /* la_prefill writes each sequence's final KV state to state_ws */
+    LA_READ_STATE = 8    /* la_prefill starts each sequence from the KV state in state_ws */
 };
 
 /* Largest number of packed sequences one la_prefill call accepts. */
@@ -72,6 +73,7 @@ enum {
  *
  *   q, k, v   [T][H][D] inputs (bf16 with LA_BF16, fp32 otherwise), T = B*N.
  *   o         [T][H][D] output, same dtype.  Every row of every sequence is written.
+ *             q, k, v and o may be NULL when there are no tokens (N == 0).
  *   B, N      without cu_seqlens: B sequences of N tokens each (B >= 1, N >= 0).
  *             With cu_seqlens: B must be 1 and N is the packed total T.
  *   H, D      heads (>= 1) and head dim; D in {64, 128}.
@@ -84,9 +86,19 @@ enum {
  *             The array is read during the call only.
  *   num_seqs  entries of cu_seqlens minus one (1 .. LA_MAX_VARLEN_SEQS); ignored
  *             when cu_seqlens is NULL.
- *   flags     LA_BF16 or LA_FP32, optionally | LA_OUT_RMSNORM | LA_WRITE_STATE.
- *   state_ws  with LA_WRITE_STATE: [S][H][D][D] fp32 (S = num_seqs or B), the
- *             final state K_s^T V_s of each sequence; otherwise ignored (may be NULL).
+ *   flags     LA_BF16 or LA_FP32, optionally | LA_OUT_RMSNORM | LA_WRITE_STATE
+ *             | LA_READ_STATE.
+ *   state_ws  [S][H][D][D] fp32 (S = num_seqs or B), used when either state flag
+ *             is set, otherwise ignored (may be NULL).
+ *             LA_READ_STATE: on entry it holds each sequence's initial state X_s,
+ *             and the sequence continues from it (chunked prefill, resume, and the
+ *             per-chunk step of LASP+, mizuki blog section 5 and appendix "key
+ *             concepts"): O_i = q_i^T X_s + sum_{j <= i in s} (q_i . k_j) v_j.
+ *             Without it every sequence starts from 0.
+ *             LA_WRITE_STATE: on exit it holds each sequence's final state,
+ *             X_s + K_s^T V_s (X_s = 0 without LA_READ_STATE).  With both flags the
+ *             update is in place: each (sequence, head) slice is read before it is
+ *             overwritten, by the same threads.
  *   stream    cudaStream_t for the launch.
  *
  * Returns LA_OK once the work is enqueued.

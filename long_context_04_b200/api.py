@@ -18,7 +18,7 @@ from . import build as _build
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA = 0, 1, 2, 3
 LA_ERR_DEVICE_TIMEOUT, LA_ERR_DEVICE_RANGE = 4, 5
-LA_FP32, LA_BF16, LA_OUT_RMSNORM, LA_WRITE_STATE = 0, 1, 2, 4
+LA_FP32, LA_BF16, LA_OUT_RMSNORM, LA_WRITE_STATE, LA_READ_STATE = 0, 1, 2, 4, 8
 LA_MAX_VARLEN_SEQS = 1024
 
 
@@ -104,13 +104,19 @@ def _flags_for(dtype) -> int:
 
 
 def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
-            return_state: bool = False, state_out=None, out=None, stream=None):
+            return_state: bool = False, state_out=None, out=None, initial_state=None,
+            stream=None):
     """Causal lightning attention over a batch (length > 1 path).
 
     ``q, k, v``: ``[B, N, H, D]`` or packed ``[T, H, D]`` (then ``cu_seqlens``,
     a host sequence of S+1 ints, gives the boundaries).  Returns ``o`` of the
-    same shape, or ``(o, state)`` with ``return_state`` (state ``[S, H, D, D]``
-    fp32, the final K^T V of each sequence).
+    same shape, or ``(o, state)`` with ``return_state`` or ``state_out`` (state
+    ``[S, H, D, D]`` fp32, the final KV of each sequence).
+
+    ``initial_state`` (``[S, H, D, D]`` fp32): each sequence continues from it
+    (chunked prefill, resume).  The final state then is ``initial + K^T V``; it
+    is written over ``initial_state`` itself when ``state_out`` is that tensor,
+    otherwise ``initial_state`` is left as it is.
     """
     _need(q, "q")
     for t, n in ((k, "k"), (v, "v")):
@@ -141,13 +147,32 @@ def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
     if st is not None:
         _need(st, "state_out", torch.float32)
         flags |= LA_WRITE_STATE
+    ws = st
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32)
+        if tuple(initial_state.shape) != (S, H, D, D):
+            raise ValueError("initial_state must be [S, H, D, D]")
+        flags |= LA_READ_STATE
+        if st is None:
+            ws = initial_state                       # read only
+        elif st.data_ptr() != initial_state.data_ptr():
+            _copy_state(initial_state, st, stream)   # the library's copy kernel; then in place
+    
     if rmsnorm:
         flags |= LA_OUT_RMSNORM
     cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
     rc = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, D, beta, cu_ptr,
-                          0 if cu is None else len(cu) - 1, flags, _ptr(st), _stream_ptr(stream))
+                          0 if cu is None else len(cu) - 1, flags, _ptr(ws), _stream_ptr(stream))
     _check("la_prefill", rc)
     return (out, st) if (return_state or state_out is not None) else out
+
+
+def _copy_state(src, dst, stream):
+    if tuple(dst.shape) != tuple(src.shape):
+        raise ValueError("state_out must have the shape of initial_state")
+    S, H, D, _ = src.shape
+    rc = lib().la_state_out(_ptr(src), _ptr(dst), S, H, D, None, S, _stream_ptr(stream))
+    _check("la_state_out", rc)
 
 
 def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None):

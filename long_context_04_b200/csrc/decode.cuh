@@ -114,4 +114,10 @@ __global__ void __launch_bounds__(256)
     for (int i = threadIdx.x; i < n4; i += blockDim.x) b[i] = __ldcs(&a[i]);
 }
 
+// dst[s][h] = 0 (the final state of sequences with no tokens); one CTA per (s, h).
+__global__ void __launch_bounds__(256) state_zero_kernel(float4 *__restrict__ dst, int n4) {
+    float4 *b = dst + (size_t)blockIdx.x * n4;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 }  // namespace la

@@ -104,13 +104,14 @@ la_status launch_pair(const la::PrefillPairParams &p, int pairs, cudaStream_t st
 
 template <int BETA, int D>
 la_status launch_simt(const float *q, const float *k, const float *v, float *o, float *state,
-                      int H, int rmsnorm, const SeqTable &seqs, int S, cudaStream_t stream) {
+                      const float *state_in, int H, int rmsnorm, const SeqTable &seqs, int S,
+                      cudaStream_t stream) {
     using C = la::SimtCfg<BETA, D>;
     auto kern = la::prefill_simt_kernel<BETA, D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
         return LA_ERR_CUDA;
-    kern<<<S * H, C::THREADS, C::SMEM_BYTES, stream>>>(q, k, v, o, state, H, rmsnorm, seqs);
+    kern<<<S * H, C::THREADS, C::SMEM_BYTES, stream>>>(q, k, v, o, state, state_in, H, rmsnorm, seqs);
     return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
@@ -136,13 +137,16 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
                      int D, int beta, const int32_t *cu_seqlens, int num_seqs, unsigned flags,
                      float *state_ws, void *stream_) {
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    const unsigned known = LA_BF16 | LA_OUT_RMSNORM | LA_WRITE_STATE;
+    const unsigned known = LA_BF16 | LA_OUT_RMSNORM | LA_WRITE_STATE | LA_READ_STATE;
     if (flags & ~known) return LA_ERR_INVALID_ARG;
     if (H < 1 || N < 0 || B < 1) return LA_ERR_INVALID_ARG;
-    if (!q || !k || !v || !o) return LA_ERR_INVALID_ARG;
+    // with no tokens (N == 0) the data pointers are never used and may be NULL
+    if (N > 0 && (!q || !k || !v || !o)) return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return LA_ERR_INVALID_ARG;
     const bool want_state = (flags & LA_WRITE_STATE) != 0;
-    if (want_state && (state_ws == nullptr || !aligned16(state_ws))) return LA_ERR_INVALID_ARG;
+    const bool read_state = (flags & LA_READ_STATE) != 0;
+    if ((want_state || read_state) && (state_ws == nullptr || !aligned16(state_ws)))
+        return LA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
     if (beta != 64 && beta != 128) return LA_ERR_UNSUPPORTED;
 
@@ -183,10 +187,20 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
 
     const int rms = (flags & LA_OUT_RMSNORM) ? 1 : 0;
     float *state = want_state ? state_ws : nullptr;
+    const float *state_in = read_state ? state_ws : nullptr;
+    if (T == 0) {
+        // Every sequence is empty: its final state is its initial state, already in
+        // place with LA_READ_STATE, else zero.
+        if (want_state && !read_state) {
+            la::state_zero_kernel<<<(unsigned)(S * H), 256, 0, stream>>>(
+                reinterpret_cast<float4 *>(state_ws), D * D / 4);
+            return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+        }
+        return LA_OK;
+    }
 
     if (flags & LA_BF16) {
-        if (T == 0 && !want_state) return LA_OK;
-        const long long Tm = T > 0 ? T : 1;  // a tensor map needs a non-empty extent
+        const long long Tm = T;
         if (beta == 128 && D == 128) {
             // paired-CTA kernel: each CTA of a pair loads half of the rows / columns
             la::PrefillPairParams pp;
@@ -196,6 +210,7 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
                 return LA_ERR_CUDA;
             pp.o = static_cast<__nv_bfloat16 *>(o);
             pp.state = state;
+            pp.state_in = state_in;
             pp.H = H;
             pp.rmsnorm = rms;
             pp.timeout_ns = kWaitLimitNs;
@@ -209,6 +224,7 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
             return LA_ERR_CUDA;
         p.o = static_cast<__nv_bfloat16 *>(o);
         p.state = state;
+        p.state_in = state_in;
         p.H = H;
         p.rmsnorm = rms;
         p.timeout_ns = kWaitLimitNs;
@@ -221,10 +237,10 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
     const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
                 *vf = static_cast<const float *>(v);
     float *of = static_cast<float *>(o);
-    if (beta == 128 && D == 128) return launch_simt<128, 128>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
-    if (beta == 64 && D == 128) return launch_simt<64, 128>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
-    if (beta == 128 && D == 64) return launch_simt<128, 64>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
-    return launch_simt<64, 64>(qf, kf, vf, of, state, H, rms, seqs, S, stream);
+    if (beta == 128 && D == 128) return launch_simt<128, 128>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
+    if (beta == 64 && D == 128) return launch_simt<64, 128>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
+    if (beta == 128 && D == 64) return launch_simt<128, 64>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
+    return launch_simt<64, 64>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
 }
 
 la_status la_decode_step(const void *q, const void *k, const void *v, float *state, void *o, int B,

@@ -54,7 +54,8 @@ struct PrefillPairParams {
     CUtensorMap tmap_k128;  // K, box 64 x 128
     CUtensorMap tmap_v128;  // V, box 64 x 128
     __nv_bfloat16 *o;
-    float *state;           // [S][H][D][D] or nullptr
+    float *state;           // [S][H][D][D] or nullptr: final states
+    const float *state_in;  // [S][H][D][D] or nullptr: initial states (may alias state)
     int H;
     int rmsnorm;
     unsigned long long timeout_ns;
@@ -139,7 +140,7 @@ struct PairMisc {
     uint64_t o_free[2];            // used in CTA 0: arrivals from both CTAs
     uint64_t dkv_free[2];
     uint64_t p_ready;
-    uint64_t snap_ready[2];        // used in CTA 0: snapshot for block j + 1 in buffer j % 2
+    uint64_t snap_ready[2];        // used in CTA 0: snapshot u (for block u) in buffer u % 2
     uint64_t drain;
     uint64_t ss_bar[2];            // group O: RMSNorm partial sums written (per block parity)
     uint32_t tmem_base;
@@ -167,6 +168,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     const int nb = (seq_len + C::BETA - 1) / C::BETA;
     // a partial last block: its value rows past the sequence end are zeroed by group P
     const bool tail = nb > 0 && seq_len < nb * C::BETA;
+    // Snapshot u of the state (bf16, buffer u % 2) feeds O_u = Q_u snap_u.  With an
+    // initial state X the first one (u = 0) is X; without one, block 0 has no
+    // inter-block term and the first snapshot is u = 1.
+    const int u0 = p.state_in != nullptr ? 0 : 1;
     const uint64_t tlimit = p.timeout_ns;
     volatile int *abort_flag = &m->abort_flag;
 
@@ -428,16 +433,16 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                     ok = false;
                     break;
                 }
-                if (b >= 1) {
-                    if (!wwait(&m->snap_ready[(b - 1) & 1], (uint32_t)(((b - 1) >> 1) & 1))) {
+                if (b >= u0) {
+                    // snapshot b is the (b - u0)/2-th use of buffer b % 2
+                    if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     if (lane == 0) {
                         const uint64_t qd = desc_kmajor_sw128(qh_addr(b));
-                        const uint64_t sd =
-                            desc_kmajor_sw128(sbase + C::OFF_SNAP + ((b - 1) & 1) * C::SNAP_BYTES);
+                        const uint64_t sd = desc_kmajor_sw128(sbase + C::OFF_SNAP + (b & 1) * C::SNAP_BYTES);
 #pragma unroll
                         for (int ks = 0; ks < C::D / 16; ++ks) {
                             const uint32_t off = (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32);
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 #pragma unroll
                     for (int ks = 0; ks < C::BETA / 16; ++ks)
                         mma_bf16_ss_pair(dO, desc_add(pd, (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32)),
-                                         desc_add(vd, ks * 2048), C::ID_PV, (b > 0 || ks > 0) ? 1u : 0u);
+                                         desc_add(vd, ks * 2048), C::ID_PV, (b >= u0 || ks > 0) ? 1u : 0u);
                     mma_commit_pair_both(&m->o_done[b % C::NDONE]);
                 }
                 __syncwarp();
@@ -543,6 +548,25 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 64; ++t) kv[t] = 0.f;
         bool ok = true;
+        // snapshot u of the state into buffer u % 2 (own 64 rows of KV^T, bf16, swizzled)
+        auto write_snap = [&](int u) {
+            const uint32_t sSnap = sbase + C::OFF_SNAP + (u & 1) * C::SNAP_BYTES;
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                st_shared_v4(sSnap + half * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4),
+                             pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
+                             pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
+                             pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
+                             pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
+            fence_proxy_async_smem();
+            arrive_leader(&m->snap_ready[u & 1]);
+        };
+        if (p.state_in != nullptr) {  // KV^T[j][i] starts at the initial state X[i][j]
+            const float *src = p.state_in + ((size_t)sid * p.H + h) * C::D * C::D + 64 * (int)cta + r;
+#pragma unroll
+            for (int t = 0; t < 64; ++t) kv[t] = src[(size_t)(64 * half + t) * C::D];
+            write_snap(0);
+        }
         for (int b = 0; b < nb; ++b) {
             // (1) state: KV^T += dKV_b^T, then the bf16 snapshot for O_{b+1} += Q_{b+1} KV
             if (!wwait(&m->kv_done[b % C::NDONE], (uint32_t)((b / C::NDONE) & 1))) {
@@ -565,18 +589,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                 }
             }
             if (b + 1 < nb) {
-                // Snapshot buffer b & 1 was last read by O_{b-1} = Q_{b-1} snap, complete
-                // since o_done(b-1), which this group waited for in the previous block.
-                const uint32_t sSnap = sbase + C::OFF_SNAP + (b & 1) * C::SNAP_BYTES;
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    st_shared_v4(sSnap + half * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4),
-                                 pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
-                                 pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
-                                 pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
-                                 pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
-                fence_proxy_async_smem();
-                arrive_leader(&m->snap_ready[b & 1]);
+                // Snapshot b + 1 goes to buffer (b+1) & 1, last read by O_{b-1} = Q_{b-1}
+                // snap_{b-1}, complete since o_done(b-1), which this group waited for in
+                // the previous block.
+                write_snap(b + 1);
             }
             // (2) output block b
             if (!wwait(&m->o_done[b % C::NDONE], (uint32_t)((b / C::NDONE) & 1))) {

@@ -28,7 +28,7 @@ template <int BETA, int D>
 __global__ void __launch_bounds__(256)
     prefill_simt_kernel(const float *__restrict__ q, const float *__restrict__ k,
                         const float *__restrict__ v, float *__restrict__ o,
-                        float *__restrict__ state, int H, int rmsnorm,
+                        float *state, const float *state_in, int H, int rmsnorm,
                         const __grid_constant__ SeqTable seqs) {
     using C = SimtCfg<BETA, D>;
     extern __shared__ float sm[];
@@ -45,7 +45,10 @@ __global__ void __launch_bounds__(256)
     int start, len, sid;
     seqs.get(rank, start, len, sid);
 
-    for (int x = tid; x < D * D; x += C::THREADS) sKV[x] = 0.f;
+    // KV starts at the sequence's initial state (state_in may alias state: this CTA
+    // reads its slice here and writes it back only at the end)
+    const float *x0 = state_in != nullptr ? state_in + ((size_t)sid * H + h) * D * D : nullptr;
+    for (int x = tid; x < D * D; x += C::THREADS) sKV[x] = x0 != nullptr ? x0[x] : 0.f;
 
     for (int p0 = 0; p0 < len; p0 += BETA) {
         const int nv = min(BETA, len - p0);

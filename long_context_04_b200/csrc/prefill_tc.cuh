@@ -70,7 +70,8 @@ struct PrefillTcParams {
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
     __nv_bfloat16 *o;
-    float *state;        // [S][H][D][D] or nullptr
+    float *state;        // [S][H][D][D] or nullptr: final states
+    const float *state_in;  // [S][H][D][D] or nullptr: initial states (may alias state)
     int H;
     int rmsnorm;
     unsigned long long timeout_ns;
@@ -131,7 +132,7 @@ struct TcMisc {
     uint64_t dkv_free[2];
     uint64_t ss_full[2];
     uint64_t p_ready;
-    uint64_t snap_ready;
+    uint64_t snap_ready[2];  // snapshot u of the state is in buffer u % 2
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -160,6 +161,10 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
     int seq_start, seq_len, sid;
     p.seqs.get(rank, seq_start, seq_len, sid);
     const int nb = (seq_len + BETA - 1) / BETA;
+    // Snapshots u of the state feed O_u += Q_u snap_u.  With an initial state X the
+    // first one (u = 0) is X itself; without one, block 0 has no inter-block term
+    // and the first snapshot is u = 1.
+    const int u0 = p.state_in != nullptr ? 0 : 1;
     const uint32_t partner = (uint32_t)(vs ^ 1);
     const uint64_t tlimit = p.timeout_ns;
     volatile int *abort_flag = &m->abort_flag;
@@ -178,7 +183,8 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             mbar_init(&m->ss_full[i], C::GROUP);
         }
         mbar_init(&m->p_ready, C::GROUP);
-        mbar_init(&m->snap_ready, C::GROUP);
+        mbar_init(&m->snap_ready[0], C::GROUP);
+        mbar_init(&m->snap_ready[1], C::GROUP);
         mbar_init(&m->drain, 1);
         m->abort_flag = 0;
         fence_mbarrier_init_cluster();
@@ -315,8 +321,10 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 mma_commit(&m->dkv_full[b & 1]);
             }
             __syncwarp();
-            if (b >= 1) {
-                if (!wwait(&m->snap_ready, (uint32_t)((b - 1) & 1))) {
+            if (b >= u0) {
+                // Snapshot b, the (b - u0)/2-th use of buffer b % 2.  One barrier per buffer:
+                // its next phase needs dKV_{b+1}, which this thread has not issued yet.
+                if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
                     ok = false;
                     break;
                 }
@@ -397,6 +405,37 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 64; ++t) kv[t] = 0.f;
         bool ok = true;
+        // snapshot u of KV into buffer u % 2 (bf16, 128-byte swizzled rows), then signal it
+        auto write_snap = [&](int u) {
+            const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (u & 1);
+            if (i_ok) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const uint32_t chunk = (uint32_t)(t ^ (i & 7));
+                    st_shared_v4(sSnap + i * 128 + (chunk << 4), pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
+                                 pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
+                                 pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
+                                 pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&m->snap_ready[u & 1]);
+        };
+        if (p.state_in != nullptr) {  // KV starts at the sequence's initial state
+            if (i_ok) {
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    p.state_in + (((size_t)sid * p.H + h) * D + i) * D + 64 * vs);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float4 x = src[t];
+                    kv[4 * t] = x.x;
+                    kv[4 * t + 1] = x.y;
+                    kv[4 * t + 2] = x.z;
+                    kv[4 * t + 3] = x.w;
+                }
+            }
+            write_snap(0);
+        }
 
         auto write_o = [&](int j) -> bool {  // read O_j out of TMEM, normalise, store
             if (!wwait(&m->o_full[j & 1], (uint32_t)((j >> 1) & 1))) return false;
@@ -469,20 +508,7 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             if (b + 1 < nb) {
                 // Buffer (b+1)&1 was last read by O_{b-1} += Q_{b-1} KV, which finished
                 // before dKV_b (MMAs complete in issue order), so it is free here.
-                const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * ((b + 1) & 1);
-                if (i_ok) {
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        const uint32_t chunk = (uint32_t)(t ^ (i & 7));
-                        st_shared_v4(sSnap + i * 128 + (chunk << 4),
-                                     pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
-                                     pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
-                                     pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
-                                     pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
-                    }
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&m->snap_ready);
+                write_snap(b + 1);
             }
             // (2) the previous block's output
             if (b >= 1 && !write_o(b - 1)) {

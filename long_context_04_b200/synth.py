@@ -52,3 +52,12 @@ def decode_tokens(B: int, H: int, D: int, step: int, seed: int = 0, dtype=torch.
     """q, k, v of shape [B, H, D] for decode step ``step`` (fresh seeded draws per step)."""
     base = 1_000_003 * (seed + 1) + 3 * step
     return tuple(normal((B, H, D), D, base + i, dtype, device) for i in range(3))
+
+
+def initial_state(S: int, H: int, D: int, tokens: int, seed: int = 0, device="cpu") -> torch.Tensor:
+    """A stand-in for the state a sequence carries after ``tokens`` earlier tokens:
+    i.i.d. N(0, 1) * sqrt(tokens) / D in fp32, shape [S, H, D, D] (the entries of a
+    sum of ``tokens`` outer products k v^T with k, v ~ N(0, 1/D) have that spread)."""
+    g = generator(7_000_003 + int(seed), device)
+    x = torch.randn((S, H, D, D), generator=g, device=device, dtype=torch.float32)
+    return x * (float(tokens) ** 0.5 / D)

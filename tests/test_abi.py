@@ -75,6 +75,9 @@ def _prefill(L, *, q=FAKE, o=FAKE, B=1, H=2, N=8, D=128, beta=128, cu=None, S=0,
     (dict(beta=256), api.LA_ERR_UNSUPPORTED),
     (dict(flags=1 | 64), api.LA_ERR_INVALID_ARG),        # unknown flag bit
     (dict(flags=1 | 4, st=None), api.LA_ERR_INVALID_ARG),  # state requested, no buffer
+    (dict(flags=1 | 8, st=None), api.LA_ERR_INVALID_ARG),  # initial state, no buffer
+    (dict(flags=1 | 4 | 8, st=FAKE + 4), api.LA_ERR_INVALID_ARG),  # misaligned state buffer
+    (dict(flags=1 | 16), api.LA_ERR_INVALID_ARG),        # unknown flag bit
     (dict(cu=[0, 3, 8], S=2, B=2), api.LA_ERR_INVALID_ARG),  # cu_seqlens needs B == 1
     (dict(cu=[1, 3, 8], S=2), api.LA_ERR_INVALID_ARG),   # must start at 0
     (dict(cu=[0, 3, 7], S=2), api.LA_ERR_INVALID_ARG),   # must end at N

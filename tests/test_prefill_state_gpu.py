@@ -1,0 +1,144 @@
+"""Prefill from an initial state (LA_READ_STATE): the CUDA path against the fp64 oracle.
+
+A sequence may continue from a state X instead of 0 (chunked prefill, resume, the
+per-chunk step of LASP+).  Cases, for every kernel family (paired bf16 beta = D = 128,
+unpaired bf16, fp32):
+  * seeded X, packed sequences with an empty one and ragged tails: outputs and final
+    states against the oracle run from the same X;
+  * a sequence run as two chunks through the library (chunk 2 from chunk 1's final
+    state) against the oracle's single run;
+  * the in-place update (state_out is initial_state) and a separate state_out that
+    leaves initial_state untouched;
+  * empty sequences return X bit for bit.
+Bounds as in the other parity tests: 1e-5 (fp32 path), 2e-2 (bf16 path), relative L2
+per (sequence, head).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_04_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
+
+# (dtype, beta, D): the paired kernel, the three unpaired bf16 shapes, the fp32 kernel
+KERNELS = [(torch.bfloat16, 128, 128), (torch.bfloat16, 64, 128), (torch.bfloat16, 128, 64),
+           (torch.bfloat16, 64, 64), (torch.float32, 128, 128), (torch.float32, 64, 64)]
+IDS = [f"{'bf16' if d == torch.bfloat16 else 'fp32'}-b{b}-d{D}" for d, b, D in KERNELS]
+
+
+def _state_err(st_gpu, st_ref):
+    worst = 0.0
+    S, H = st_ref.shape[:2]
+    for s in range(S):
+        for h in range(H):
+            worst = max(worst, oracle.rel_l2(st_gpu[s, h], st_ref[s, h]))
+    return worst
+
+
+@pytest.mark.parametrize("dtype,beta,D", KERNELS, ids=IDS)
+@pytest.mark.parametrize("rmsnorm", [False, True], ids=["plain", "rmsnorm"])
+def test_seeded_initial_state(dtype, beta, D, rmsnorm):
+    H = 3
+    cu = [0, 300, 300, 700, 829]            # lengths 300, 0, 400, 129
+    T, S = cu[-1], len(cu) - 1
+    q, k, v = synth.qkv(T, H, D, seed=31, dtype=dtype, device="cuda")
+    x = synth.initial_state(S, H, D, tokens=2000, seed=31, device="cuda")
+    x_host = x.cpu().numpy()
+    o, st = api.prefill(q, k, v, beta=beta, cu_seqlens=cu, rmsnorm=rmsnorm, initial_state=x,
+                        return_state=True)
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LA_OK
+    ref_o, ref_s = oracle.recurrent(q, k, v, cu, rmsnorm=rmsnorm, initial_state=x_host)
+    assert oracle.max_rel_l2_per_head(o, ref_o, cu) <= TOL[dtype]
+    assert _state_err(st.cpu().numpy(), ref_s) <= (1e-6 if dtype == torch.float32 else 1e-5)
+    # the empty sequence keeps X exactly, and X itself was not written
+    assert torch.equal(st[1], x[1])
+    assert np.array_equal(x.cpu().numpy(), x_host)
+
+
+@pytest.mark.parametrize("dtype,beta,D", KERNELS, ids=IDS)
+@pytest.mark.parametrize("cut", [0, 1, 128, 517, 1000], ids=lambda c: f"cut{c}")
+def test_two_chunks_equal_one_run(dtype, beta, D, cut):
+    """Chunk 2 continues from the state the library wrote for chunk 1."""
+    H, T = 2, 1000
+    q, k, v = synth.qkv(T, H, D, seed=32, dtype=dtype, device="cuda")
+    o = torch.empty_like(q)   # chunk outputs are views of it (an empty chunk still has an address)
+    _, st = api.prefill(q[:cut], k[:cut], v[:cut], beta=beta, return_state=True, out=o[:cut])
+    api.prefill(q[cut:], k[cut:], v[cut:], beta=beta, initial_state=st, state_out=st,  # in place
+                out=o[cut:])
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LA_OK
+    ref_o, ref_s = oracle.recurrent(q, k, v)
+    assert oracle.max_rel_l2_per_head(o, ref_o) <= TOL[dtype]
+    assert _state_err(st.cpu().numpy(), ref_s) <= (1e-6 if dtype == torch.float32 else 1e-5)
+
+
+@pytest.mark.parametrize("dtype,beta,D", KERNELS[:2] + KERNELS[4:5], ids=IDS[:2] + IDS[4:5])
+def test_packed_chunks_with_state(dtype, beta, D):
+    """Several packed sequences, each cut in two; chunk 2 of all of them runs packed
+    from the chunk-1 states."""
+    H = 2
+    lens = [257, 0, 640, 31]
+    cuts = [100, 0, 384, 31]
+    q, k, v = synth.qkv(sum(lens), H, D, seed=33, dtype=dtype, device="cuda")
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    rows1 = np.concatenate([np.arange(starts[s], starts[s] + cuts[s]) for s in range(4)])
+    rows2 = np.concatenate([np.arange(starts[s] + cuts[s], starts[s + 1]) for s in range(4)])
+    cu1 = np.concatenate([[0], np.cumsum(cuts)]).tolist()
+    cu2 = np.concatenate([[0], np.cumsum(np.array(lens) - np.array(cuts))]).tolist()
+    r1, r2 = torch.as_tensor(rows1, device="cuda"), torch.as_tensor(rows2, device="cuda")
+    o1, st1 = api.prefill(q[r1], k[r1], v[r1], beta=beta, cu_seqlens=cu1, return_state=True)
+    o2, st2 = api.prefill(q[r2], k[r2], v[r2], beta=beta, cu_seqlens=cu2, initial_state=st1,
+                          return_state=True)              # separate state_out
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LA_OK
+    cu = starts.tolist()
+    ref_o, ref_s = oracle.recurrent(q, k, v, cu)
+    o = torch.empty_like(q)
+    o[r1], o[r2] = o1, o2
+    assert oracle.max_rel_l2_per_head(o, ref_o, cu) <= TOL[dtype]
+    assert _state_err(st2.cpu().numpy(), ref_s) <= (1e-6 if dtype == torch.float32 else 1e-5)
+    # st1 (the initial state of chunk 2) is left as it was: it is K^T V of chunk 1
+    ref_s1 = oracle.final_state(k[r1], v[r1], cu1)
+    assert _state_err(st1.cpu().numpy(), ref_s1) <= (1e-6 if dtype == torch.float32 else 1e-5)
+
+
+@pytest.mark.parametrize("dtype,beta,D", KERNELS, ids=IDS)
+def test_all_empty_sequences_keep_state(dtype, beta, D):
+    H = 2
+    q = torch.zeros((4, H, D), dtype=dtype, device="cuda")
+    x = synth.initial_state(3, H, D, tokens=100, seed=34, device="cuda")
+    # empty sequences mixed with a non-empty one, then all empty (no launch at all)
+    st = x.clone()
+    api.prefill(q, q, q, beta=beta, cu_seqlens=[0, 0, 4, 4], initial_state=st, state_out=st,
+                out=torch.empty_like(q))
+    torch.cuda.synchronize()
+    assert torch.equal(st[0], x[0]) and torch.equal(st[2], x[2])
+    st = x.clone()
+    e = q[:0]
+    api.prefill(e, e, e, beta=beta, cu_seqlens=[0, 0, 0, 0], initial_state=st, state_out=st,
+                out=torch.empty_like(q)[:0])
+    torch.cuda.synchronize()
+    assert torch.equal(st, x)
+    assert api.device_status() == api.LA_OK
+
+
+def test_long_paired_sequence_with_state_sampled_heads():
+    """The paired kernel over many blocks from a large initial state: two sampled heads
+    against the oracle, every head's final state against the oracle's X + K^T V."""
+    N, H, D = 16384, 8, 128
+    q, k, v = synth.qkv(N, H, D, seed=35, dtype=torch.bfloat16, device="cuda")
+    x = synth.initial_state(1, H, D, tokens=100000, seed=35, device="cuda")
+    o, st = api.prefill(q, k, v, beta=128, initial_state=x, return_state=True)
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LA_OK
+    heads = [0, 5]
+    ref_o, _ = oracle.recurrent(q[:, heads], k[:, heads], v[:, heads],
+                                initial_state=x[:, heads].cpu().numpy())
+    assert oracle.max_rel_l2_per_head(o[:, heads], ref_o) <= 2e-2
+    ref_s = x.cpu().double().numpy() + oracle.final_state(k, v)
+    assert _state_err(st.cpu().numpy(), ref_s) <= 1e-5
