@@ -17,9 +17,8 @@
 // so a CTA stages only its halves (64 KB per block instead of 80 KB for the
 // unpaired kernel) and each tensor-core operand byte is read once per pair
 // instead of once per CTA.  The halves arrive through three TMA rings (key
-// rows 2 deep, query rows 4 deep, key dims + value columns 3 deep), each slot
-// released at the last MMA that reads it, so every load has about two blocks
-// of time to land.  Each CTA keeps
+// rows 2 deep, query rows 4 deep, key dims + value columns 2 deep), each slot
+// released by the last MMA that reads it.  Each CTA keeps
 // its 64 columns of the fp32 state, transposed (KV^T[j][i]), in epilogue
 // registers, and its output rows are complete (all 128 columns) inside the
 // CTA, so the RMSNorm needs no exchange between the CTAs.
@@ -62,17 +61,20 @@ struct PrefillPairParams {
     SeqTable seqs;
 };
 
-#ifndef LA_PAIR_DKV_FIRST
-#define LA_PAIR_DKV_FIRST 1
+#ifndef LA_PAIR_S_AHEAD
+#define LA_PAIR_S_AHEAD 1
+#endif
+#ifndef LA_PAIR_P_BUFS
+#define LA_PAIR_P_BUFS 1
 #endif
 #ifndef LA_PAIR_KK_DEPTH
 #define LA_PAIR_KK_DEPTH 2
 #endif
 #ifndef LA_PAIR_QH_DEPTH
-#define LA_PAIR_QH_DEPTH 3
+#define LA_PAIR_QH_DEPTH 4
 #endif
 #ifndef LA_PAIR_KV_DEPTH
-#define LA_PAIR_KV_DEPTH 3
+#define LA_PAIR_KV_DEPTH 2
 #endif
 
 struct PairCfg {
@@ -88,24 +90,31 @@ struct PairCfg {
     // ring of block-completion barriers; a ring's depth may not exceed the barrier
     // ring it waits on, or a phase could be lapped before its waiter sees it
     static constexpr int NDONE = 4;
-    static_assert(NKK == 2, "key-row slots are released by s_full[2]");
+    // S runs SAHEAD blocks ahead of the block whose P V consumes it, in a ring of
+    // SAHEAD + 1 TMEM buffers (the extra one is being turned into P by group P)
+    static constexpr int SAHEAD = LA_PAIR_S_AHEAD, NS = SAHEAD + 1;
+    static_assert(NKK <= NS, "key-row slots are released by s_full[NS]");
     static_assert(NQH <= NDONE && NKV <= NDONE, "slot release ring");
     static constexpr int KK_BYTES = 2 * HBOX, QH_BYTES = 2 * HBOX, KV_BYTES = 2 * FBOX;
     static constexpr int OFF_KK = 0;
     static constexpr int OFF_QH = OFF_KK + NKK * KK_BYTES;
     static constexpr int OFF_KV = OFF_QH + NQH * QH_BYTES;
     static constexpr int KV_OFF_VC = FBOX;               // within a KV stage
-    static constexpr int OFF_P = OFF_KV + NKV * KV_BYTES;  // own 64 rows of P, keys [0,64) | [64,128)
+    // P buffers (own 64 rows of P, keys [0,64) | [64,128)); P_b goes to buffer b % NPB
+    static constexpr int NPB = LA_PAIR_P_BUFS, P_BYTES = 2 * HBOX;
+    static_assert(NPB <= NDONE, "P buffers are released by o_done");
+    static constexpr int OFF_P = OFF_KV + NKV * KV_BYTES;
     // two bf16 snapshots of the state (own 64 rows of KV^T, dims [0,64) | [64,128)):
     // the one for block b+1 is written while O_b = Q_b snap still reads the other
     static constexpr int SNAP_BYTES = 2 * HBOX;
-    static constexpr int OFF_SNAP = OFF_P + 2 * HBOX;
+    static constexpr int OFF_SNAP = OFF_P + NPB * P_BYTES;
     static constexpr int OFF_MISC = OFF_SNAP + 2 * SNAP_BYTES;
     static constexpr int MISC = 2048;
     static constexpr int SMEM_BYTES = 1024 + OFF_MISC + MISC;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-    // TMEM columns: S[2], O[2], dKV[2], 64 columns each (folded layout)
-    static constexpr int TM_S = 0, TM_O = 128, TM_DKV = 256;
+    // TMEM columns: S[NS], O[2], dKV[2], 64 columns each (folded layout)
+    static constexpr int TM_S = 0, TM_O = 64 * NS, TM_DKV = 64 * NS + 128;
+    static_assert(TM_DKV + 128 <= 512, "TMEM columns");
     static constexpr int TMEM_COLS = 512;
     static constexpr int GROUP = 128;
     static constexpr int WARP_B = 10;                   // second MMA issuer (CTA 0)
@@ -119,12 +128,12 @@ struct PairCfg {
 // Every wait below is a parity wait on one phase x of a barrier.  Two rules make
 // it exact: phase x - 1 is known to be complete when the wait starts (the waiter
 // saw it, or a chain of signals implies it), and phase x + 1 cannot complete
-// before the wait returns.  This is why the S buffers and the snapshots have a
-// release barrier per buffer and the tail zeroing a single-phase barrier.
+// before the wait returns.  This is why the S buffers, the P buffers and the
+// snapshots have a barrier per buffer and the tail zeroing a single-phase barrier.
 struct PairMisc {
     // Ring barriers.  "full" barriers are used in CTA 0 only: CTA 0's producer
     // expects the bytes of both CTAs and CTA 1's loads complete them directly.
-    // A slot is free again once the MMAs reading it have completed: s_full[j % 2]
+    // A slot is free again once the MMAs reading it have completed: s_full[j % NS]
     // frees key-row slot j (S_j done), o_done[j % 4] the query slot (O_j done, which
     // follows S_j), o_done and kv_done[j % 4] together the K/V slot.  Every MMA
     // commit arrives on the barrier of both CTAs.
@@ -133,13 +142,13 @@ struct PairMisc {
     uint64_t full_kv[PairCfg::NKV];
     uint64_t tail_kv;              // CTA 1: its own KV tiles of a partial last block landed
     uint64_t tail_zeroed;          // used in CTA 0: value rows past the sequence end zeroed
-    uint64_t s_full[2];            // S_j complete
-    uint64_t s_free[2];            // used in CTA 0: group P of both CTAs has loaded S_j
+    uint64_t s_full[PairCfg::NS];  // S_j complete (buffer j % NS)
+    uint64_t s_free[PairCfg::NS];  // used in CTA 0: group P of both CTAs has loaded S_j
     uint64_t kv_done[4];           // dKV_j complete (issuer A)
     uint64_t o_done[4];            // O_j complete (issuer B)
     uint64_t o_free[2];            // used in CTA 0: arrivals from both CTAs
     uint64_t dkv_free[2];
-    uint64_t p_ready;
+    uint64_t p_ready[PairCfg::NPB];  // used in CTA 0: P_j stored in buffer j % NPB
     uint64_t snap_ready[2];        // used in CTA 0: snapshot u (for block u) in buffer u % 2
     uint64_t drain;
     uint64_t ss_bar[2];            // group O: RMSNorm partial sums written (per block parity)
@@ -179,6 +188,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         for (int s = 0; s < C::NKK; ++s) mbar_init(&m->full_kk[s], 1);
         for (int s = 0; s < C::NQH; ++s) mbar_init(&m->full_qh[s], 1);
         for (int s = 0; s < C::NKV; ++s) mbar_init(&m->full_kv[s], 1);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&m->s_full[s], 1);
+            mbar_init(&m->s_free[s], 2 * C::GROUP);
+        }
         for (int s = 0; s < C::NDONE; ++s) {
             mbar_init(&m->kv_done[s], 1);
             mbar_init(&m->o_done[s], 1);
@@ -186,13 +199,11 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         mbar_init(&m->tail_kv, 1);
         mbar_init(&m->tail_zeroed, 2 * C::GROUP);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&m->s_full[i], 1);
-            mbar_init(&m->s_free[i], 2 * C::GROUP);
             mbar_init(&m->snap_ready[i], 2 * C::GROUP);
             mbar_init(&m->o_free[i], 2 * C::GROUP);
             mbar_init(&m->dkv_free[i], 2 * C::GROUP);
         }
-        mbar_init(&m->p_ready, 2 * C::GROUP);
+        for (int i = 0; i < C::NPB; ++i) mbar_init(&m->p_ready[i], 2 * C::GROUP);
         mbar_init(&m->drain, 2);
         mbar_init(&m->ss_bar[0], C::GROUP);
         mbar_init(&m->ss_bar[1], C::GROUP);
@@ -269,7 +280,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             uint32_t polls = 0;
             while (jk < nb || jq < nb || jv < nb) {
                 bool progressed = false;
-                if (jk < nb && freed(m->s_full, 2, jk, C::NKK)) {
+                if (jk < nb && freed(m->s_full, C::NS, jk, C::NKK)) {
                     uint64_t *fb = &m->full_kk[jk % C::NKK];
                     const uint32_t dst = kk_addr(jk);
                     const int row = seq_start + jk * C::BETA + own_rows;
@@ -362,8 +373,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             if (!wwait(&m->full_kk[j % C::NKK], (uint32_t)((j / C::NKK) & 1)) ||
                 !wwait(&m->full_qh[j % C::NQH], (uint32_t)((j / C::NQH) & 1)))
                 return false;
-            // S buffer j & 1 was last read by group P for block j - 2
-            if (j >= 2 && !wwait(&m->s_free[j & 1], (uint32_t)(((j - 2) >> 1) & 1))) return false;
+            // S buffer j % NS was last read by group P for block j - NS
+            if (j >= C::NS && !wwait(&m->s_free[j % C::NS], (uint32_t)(((j - C::NS) / C::NS) & 1)))
+                return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t qd = desc_kmajor_sw128(qh_addr(j));
@@ -371,23 +383,20 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 #pragma unroll
                 for (int ks = 0; ks < C::D / 16; ++ks) {
                     const uint32_t off = (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32);
-                    mma_bf16_ss_pair(tmem + C::TM_S + 64 * (j & 1), desc_add(qd, off),
+                    mma_bf16_ss_pair(tmem + C::TM_S + 64 * (j % C::NS), desc_add(qd, off),
                                      desc_add(kd, off), C::ID_S, ks > 0 ? 1u : 0u);
                 }
-                mma_commit_pair_both(&m->s_full[j & 1]);
+                mma_commit_pair_both(&m->s_full[j % C::NS]);
             }
             __syncwarp();
             return true;
         };
-        // Per block b: dKV_b^T = V_b^T K_b, then S_{b+1} (look-ahead, so that group P has a
-        // block's time to form P_{b+1}).  dKV_b goes first: the snapshot of KV_{<b+1} that
-        // issuer B waits for is derived from it.
-        bool ok = nb == 0 || stage_in(0);
+        // Per block b: dKV_b^T = V_b^T K_b, then S_{b+SAHEAD} (look-ahead, so that group P
+        // has SAHEAD blocks' time to form P from it).  dKV_b goes first: the snapshot of
+        // KV_{<b+1} that issuer B waits for is derived from it.
+        bool ok = true;
+        for (int j = 0; ok && j < C::SAHEAD && j < nb; ++j) ok = stage_in(j);
         for (int b = 0; ok && b < nb; ++b) {
-            if (!LA_PAIR_DKV_FIRST && b + 1 < nb && !stage_in(b + 1)) {
-                ok = false;
-                break;
-            }
             const uint32_t kva = kv_addr(b);
             // a partial last block: group P zeroes the value rows past the sequence end
             // before dKV_b may read them
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                 mma_commit_pair_both(&m->kv_done[b % C::NDONE]);
             }
             __syncwarp();
-            if (LA_PAIR_DKV_FIRST && b + 1 < nb && !stage_in(b + 1)) {
+            if (b + C::SAHEAD < nb && !stage_in(b + C::SAHEAD)) {
                 ok = false;
                 break;
             }
@@ -429,7 +438,11 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             bool ok = true;
             for (int b = 0; ok && b < nb; ++b) {
                 const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
-                if (b >= 2 && !wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1))) {
+                // The query tile of block b must have landed: nothing else that this thread
+                // waits for implies it (S_b was issued by the other thread, and the
+                // snapshot does not depend on it).  Checked for every block, in order.
+                if ((b >= 2 && !wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1))) ||
+                    !wwait(&m->full_qh[b % C::NQH], (uint32_t)((b / C::NQH) & 1))) {
                     ok = false;
                     break;
                 }
@@ -452,14 +465,14 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                     }
                     __syncwarp();
                 }
-                if (!wwait(&m->p_ready, (uint32_t)(b & 1)) ||
+                if (!wwait(&m->p_ready[b % C::NPB], (uint32_t)((b / C::NPB) & 1)) ||
                     !wwait(&m->full_kv[b % C::NKV], (uint32_t)((b / C::NKV) & 1))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint64_t pd = desc_kmajor_sw128(sbase + C::OFF_P);
+                    const uint64_t pd = desc_kmajor_sw128(sbase + C::OFF_P + (b % C::NPB) * C::P_BYTES);
                     const uint64_t vd = desc_mnmajor_sw128(kv_addr(b) + C::KV_OFF_VC, C::FBOX);
 #pragma unroll
                     for (int ks = 0; ks < C::BETA / 16; ++ks)
@@ -486,18 +499,18 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         const uint32_t sP = sbase + C::OFF_P;
         bool ok = true;
         for (int b = 0; b < nb; ++b) {
-            if (!wwait(&m->s_full[b & 1], (uint32_t)((b >> 1) & 1))) {
+            if (!wwait(&m->s_full[b % C::NS], (uint32_t)((b / C::NS) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t s0[32], s1[32];
-            const uint32_t tS = tmem + C::TM_S + 64 * (b & 1) + lane_base;
+            const uint32_t tS = tmem + C::TM_S + 64 * (b % C::NS) + lane_base;
             tmem_ld32(tS, s0);
             tmem_ld32(tS + 32, s1);
             tmem_ld_wait();
             tc_fence_before();
-            arrive_leader_free(&m->s_free[b & 1]);
+            arrive_leader_free(&m->s_free[b % C::NS]);
             uint32_t w[32];
 #pragma unroll
             for (int u = 0; u < 32; ++u) {
@@ -507,14 +520,15 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                 const float x1 = c0 + 1 <= R ? __uint_as_float(s[1]) : 0.f;
                 w[u] = pack_bf16x2(x0, x1);
             }
-            // the previous block's O += P V must have read P before it is overwritten
-            if (b >= 1 && !wwait(&m->o_done[(b - 1) % C::NDONE], (uint32_t)(((b - 1) / C::NDONE) & 1))) {
+            // P buffer b % NPB was last read by O_{b-NPB} += P V; that must be complete
+            const int pb = b - C::NPB;
+            if (pb >= 0 && !wwait(&m->o_done[pb % C::NDONE], (uint32_t)((pb / C::NDONE) & 1))) {
                 ok = false;
                 break;
             }
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-                st_shared_v4(sP + kh * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4), w[4 * t],
+                st_shared_v4(sP + (b % C::NPB) * C::P_BYTES + kh * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4), w[4 * t],
                              w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
             // V rows past the sequence end must not enter dKV^T: zero them in this CTA's
             // slice once its KV tiles of the block have landed.
@@ -535,7 +549,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            arrive_leader(&m->p_ready);
+            arrive_leader(&m->p_ready[b % C::NPB]);
         }
         if (!ok) fail();
     } else {

@@ -133,12 +133,15 @@ def test_long_paired_sequence_with_state_sampled_heads():
     N, H, D = 16384, 8, 128
     q, k, v = synth.qkv(N, H, D, seed=35, dtype=torch.bfloat16, device="cuda")
     x = synth.initial_state(1, H, D, tokens=100000, seed=35, device="cuda")
-    o, st = api.prefill(q, k, v, beta=128, initial_state=x, return_state=True)
-    torch.cuda.synchronize()
-    assert api.device_status() == api.LA_OK
     heads = [0, 5]
     ref_o, _ = oracle.recurrent(q[:, heads], k[:, heads], v[:, heads],
                                 initial_state=x[:, heads].cpu().numpy())
-    assert oracle.max_rel_l2_per_head(o[:, heads], ref_o) <= 2e-2
     ref_s = x.cpu().double().numpy() + oracle.final_state(k, v)
-    assert _state_err(st.cpu().numpy(), ref_s) <= 1e-5
+    # repeated: with 16 CTAs the loads land fast or slow relative to the MMAs from run to
+    # run, which is what exposed an unguarded operand read once
+    for _ in range(3):
+        o, st = api.prefill(q, k, v, beta=128, initial_state=x, return_state=True)
+        torch.cuda.synchronize()
+        assert api.device_status() == api.LA_OK
+        assert oracle.max_rel_l2_per_head(o[:, heads], ref_o) <= 2e-2
+        assert _state_err(st.cpu().numpy(), ref_s) <= 1e-5
