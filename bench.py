@@ -387,7 +387,9 @@ def run_ours(args):
 
     if not args.no_extras:
         line["e2e"] = e2e_prefill(args, api, torch, q, k, v, B, N, H, D, beta, world, dev)
-        line["decode"] = bench_decode(api, synth, torch, dev, stream, peak_bw, rank, world)
+        line["decode"], dctx = bench_decode(api, synth, torch, dev, stream, peak_bw, rank, world)
+        line["concurrent"] = bench_concurrent(api, torch, stream, dctx, q, k, v, o, beta, world)
+        del dctx
     if rank == 0 and not args.no_extras:
         line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
     if world > 1:
@@ -473,12 +475,49 @@ def bench_decode(api, synth, torch, dev, pstream, peak_bw, rank, world):
     total_ms = dist_max(ev[0].elapsed_time(ev[steps]), world, dev)
     gbs = decode_bytes(B, H, D) / (med_ms / 1e3) / 1e9
     status = api.device_status(dstream)
-    return {"workload": f"decode step, B={B}, H={H}, D={D}, bf16 q/k/v/o, fp32 state from a "
-                        f"seeded N={N} prefill, {steps} consecutive steps",
-            "tokens_per_s": B * world * steps / (total_ms / 1e3),
-            "ms_per_step_median": med_ms, "gbs_median_step": gbs, "pct_hbm": 100.0 * gbs / peak_bw,
-            "bytes_per_step": decode_bytes(B, H, D), "gpu_launches": steps,
-            "status": api.status_string(status), "stream": "own stream (not the prefill stream)"}
+    res = {"workload": f"decode step, B={B}, H={H}, D={D}, bf16 q/k/v/o, fp32 state from a "
+                       f"seeded N={N} prefill, {steps} consecutive steps",
+           "tokens_per_s": B * world * steps / (total_ms / 1e3),
+           "ms_per_step_median": med_ms, "gbs_median_step": gbs, "pct_hbm": 100.0 * gbs / peak_bw,
+           "bytes_per_step": decode_bytes(B, H, D), "gpu_launches": steps,
+           "status": api.status_string(status), "stream": "own stream (not the prefill stream)"}
+    return res, (dstream, state, toks, outs)
+
+
+def bench_concurrent(api, torch, pstream, dctx, q, k, v, o, beta, world, n_prefill=2):
+    """The two paths together, as the pages arrange them (length-1 and length>1 requests on
+    two streams): the main prefill workload on its stream while the decode steps run on
+    theirs.  Each was also measured alone above."""
+    dstream, state, toks, outs = dctx
+    steps = len(toks)
+    ea = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    eb = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    ea[0].record(pstream)
+    for _ in range(n_prefill):
+        api.prefill(q, k, v, beta=beta, out=o, stream=pstream)
+    ea[1].record(pstream)
+    eb[0].record(dstream)
+    for t in range(steps):
+        api.decode_step(*toks[t], state, out=outs[t], stream=dstream)
+        eb[t + 1].record(dstream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    status = api.device_status(pstream)
+    per = [eb[t].elapsed_time(eb[t + 1]) for t in range(steps)]
+    first = ea[0] if ea[0].elapsed_time(eb[0]) >= 0 else eb[0]
+    last = ea[1] if eb[steps].elapsed_time(ea[1]) >= 0 else eb[steps]
+    overlapped = sum(1 for t in range(steps) if eb[t].elapsed_time(ea[1]) > 0)
+    return {"prefill_ms_per_launch": ea[0].elapsed_time(ea[1]) / n_prefill,
+            "prefill_launches": n_prefill, "decode_steps": steps,
+            "decode_steps_started_during_prefill": overlapped,
+            "decode_ms_per_step_median": statistics.median(per),
+            "decode_ms_per_step_max": max(per),
+            "span_ms": first.elapsed_time(last),
+            "status": api.status_string(status),
+            "note": "prefill on one stream and the decode steps on another, enqueued together; "
+                    "the prefill's persistent CTA pairs hold 128 of the 148 SMs while it runs"}
 
 
 def run_decode_small(args):

@@ -109,6 +109,40 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o,
                      unsigned flags, float *state_ws, void *stream);
 
 /*
+ * la_chunk_state -- each sequence's state K_s^T V_s alone, without the attention
+ * output: the local state of one chunk in LASP+, the sequence-parallel scheme the
+ * pages name for lightning attention (mizuki blog, section 5 "pretraining" and
+ * appendix "key concepts": local prefix sums of the chunk states, an all-gather,
+ * then each chunk runs from the sum of the states before it).
+ *
+ *   k, v      [T][H][D] (bf16 with LA_BF16, else fp32), T = B*N; may be NULL when
+ *             N == 0.
+ *   B, N, H, D, cu_seqlens, num_seqs
+ *             as for la_prefill (D in {64, 128}).
+ *   flags     LA_BF16 or LA_FP32; no other bit.
+ *   state_out [S][H][D][D] fp32: state_out[s][h][i][j] = sum_{t in s} k_t[i] v_t[j]
+ *             (0 for an empty sequence).  Written, never read.
+ *   stream    cudaStream_t for the launch.
+ */
+la_status la_chunk_state(const void *k, const void *v, int B, int H, int N, int D,
+                         const int32_t *cu_seqlens, int num_seqs, unsigned flags,
+                         float *state_out, void *stream);
+
+/*
+ * la_state_prefix -- the initial state of chunk `rank` in LASP+, from the chunk
+ * states of all R ranks (as an all-gather lays them out):
+ *     out[s][h] = sum_{r < rank} gathered[r][s][h]      (0 for rank 0),
+ * summed in fp32 in ascending r, so every rank adds in the same order.
+ *
+ *   gathered  [R][S][H][D][D] fp32, rank-major.
+ *   R         number of chunks (>= 1); rank in 0 .. R (rank = R gives the state
+ *             after the whole sequence).
+ *   out       [S][H][D][D] fp32; must not overlap gathered.
+ */
+la_status la_state_prefix(const float *gathered, int R, int rank, int S, int H, int D,
+                          float *out, void *stream);
+
+/*
  * la_decode_step -- one token per sequence (length-1 path).
  *
  *   q, k, v   [B][H][D] the new token's projections (bf16 with LA_BF16, else fp32).

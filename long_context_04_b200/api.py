@@ -58,6 +58,10 @@ def lib() -> ctypes.CDLL:
     L.la_decode_step.restype = i32
     L.la_state_out.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp]
     L.la_state_out.restype = i32
+    L.la_chunk_state.argtypes = [vp, vp, i32, i32, i32, i32, ip, i32, u32, vp, vp]
+    L.la_chunk_state.restype = i32
+    L.la_state_prefix.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp]
+    L.la_state_prefix.restype = i32
     L.la_status_string.argtypes = [i32]
     L.la_status_string.restype = ctypes.c_char_p
     L.la_get_device_status.argtypes = [vp]
@@ -210,6 +214,49 @@ def state_out(state_ws, state_dst, seq_to_slot=None, *, stream=None):
                             state_dst.shape[0], _stream_ptr(stream))
     _check("la_state_out", rc)
     return state_dst
+
+
+def chunk_state(k, v, *, cu_seqlens=None, state_out=None, stream=None):
+    """Each sequence's K^T V alone (no output): ``[S, H, D, D]`` fp32.  The local state
+    of a chunk in LASP+ sequence parallelism."""
+    _need(k, "k")
+    _need(v, "v", k.dtype)
+    if v.shape != k.shape:
+        raise ValueError("k and v must have one shape")
+    flags = _flags_for(k.dtype)
+    if k.dim() == 4:
+        B, N, H, D = k.shape
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens needs packed [T, H, D] inputs")
+        S = B
+    elif k.dim() == 3:
+        T, H, D = k.shape
+        B, N = 1, T
+        S = 1 if cu_seqlens is None else len(cu_seqlens) - 1
+    else:
+        raise ValueError("k must be [B, N, H, D] or [T, H, D]")
+    cu = None if cu_seqlens is None else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    if state_out is None:
+        state_out = torch.empty((S, H, D, D), dtype=torch.float32, device=k.device)
+    _need(state_out, "state_out", torch.float32)
+    cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    rc = lib().la_chunk_state(_ptr(k), _ptr(v), B, H, N, D, cu_ptr, 0 if cu is None else len(cu) - 1,
+                              flags, _ptr(state_out), _stream_ptr(stream))
+    _check("la_chunk_state", rc)
+    return state_out
+
+
+def state_prefix(gathered, rank: int, *, out=None, stream=None):
+    """``out = sum_{r < rank} gathered[r]`` for gathered ``[R, S, H, D, D]`` fp32 (the
+    chunk states of all ranks): the initial state of chunk ``rank`` in LASP+."""
+    _need(gathered, "gathered", torch.float32)
+    R, S, H, D, _ = gathered.shape
+    if out is None:
+        out = torch.empty((S, H, D, D), dtype=torch.float32, device=gathered.device)
+    _need(out, "out", torch.float32)
+    rc = lib().la_state_prefix(_ptr(gathered), R, int(rank), S, H, D, _ptr(out), _stream_ptr(stream))
+    _check("la_state_prefix", rc)
+    return out
 
 
 def device_status(stream=None) -> int:

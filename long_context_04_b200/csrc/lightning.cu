@@ -2,7 +2,8 @@
 //
 // Host side only: argument validation, the sequence table, TMA tensor maps and
 // kernel launches.  Every step of the computation runs in the kernels of
-// prefill_tc.cuh (bf16, tcgen05), prefill_simt.cuh (fp32), decode.cuh.
+// prefill_pair.cuh and prefill_tc.cuh (bf16, tcgen05), prefill_simt.cuh (fp32),
+// chunk_state.cuh and decode.cuh.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -10,6 +11,7 @@
 #include <numeric>
 #include <vector>
 
+#include "chunk_state.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_pair.cuh"
@@ -57,6 +59,44 @@ bool make_map(CUtensorMap *map, const void *base, long long T, int H, int D, int
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
+}
+
+// The sequence table of a call: B equal sequences of N tokens, or the packed
+// boundaries cu_seqlens (host array, validated here), ordered longest first so
+// that the block scheduler starts the longest chains first.
+la_status build_seq_table(int B, int N, const int32_t *cu_seqlens, int num_seqs, SeqTable &seqs,
+                          long long &T, int &S) {
+    std::memset(&seqs, 0, sizeof seqs);
+    T = 0;
+    S = 0;
+    if (cu_seqlens != nullptr) {
+        if (B != 1) return LA_ERR_INVALID_ARG;
+        if (num_seqs < 1) return LA_ERR_INVALID_ARG;
+        if (num_seqs > LA_MAX_VARLEN_SEQS) return LA_ERR_UNSUPPORTED;
+        if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != N) return LA_ERR_INVALID_ARG;
+        for (int s = 0; s < num_seqs; ++s)
+            if (cu_seqlens[s + 1] < cu_seqlens[s]) return LA_ERR_INVALID_ARG;
+        S = num_seqs;
+        T = N;
+        std::vector<int> order(S);
+        std::iota(order.begin(), order.end(), 0);
+        std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+            return cu_seqlens[a + 1] - cu_seqlens[a] > cu_seqlens[b + 1] - cu_seqlens[b];
+        });
+        seqs.varlen = 1;
+        for (int r = 0; r < S; ++r) {
+            const int s = order[r];
+            seqs.seq_start[r] = cu_seqlens[s];
+            seqs.seq_len[r] = cu_seqlens[s + 1] - cu_seqlens[s];
+            seqs.seq_id[r] = s;
+        }
+    } else {
+        S = B;
+        T = (long long)B * N;
+        seqs.varlen = 0;
+        seqs.N = N;
+    }
+    return LA_OK;
 }
 
 template <int BETA, int D>
@@ -152,36 +192,10 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
 
     // Sequence table (host-validated).
     SeqTable seqs;
-    std::memset(&seqs, 0, sizeof seqs);
     long long T = 0;
     int S = 0;
-    if (cu_seqlens != nullptr) {
-        if (B != 1) return LA_ERR_INVALID_ARG;
-        if (num_seqs < 1) return LA_ERR_INVALID_ARG;
-        if (num_seqs > LA_MAX_VARLEN_SEQS) return LA_ERR_UNSUPPORTED;
-        if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != N) return LA_ERR_INVALID_ARG;
-        for (int s = 0; s < num_seqs; ++s)
-            if (cu_seqlens[s + 1] < cu_seqlens[s]) return LA_ERR_INVALID_ARG;
-        S = num_seqs;
-        T = N;
-        std::vector<int> order(S);
-        std::iota(order.begin(), order.end(), 0);
-        std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-            return cu_seqlens[a + 1] - cu_seqlens[a] > cu_seqlens[b + 1] - cu_seqlens[b];
-        });
-        seqs.varlen = 1;
-        for (int r = 0; r < S; ++r) {
-            const int s = order[r];
-            seqs.seq_start[r] = cu_seqlens[s];
-            seqs.seq_len[r] = cu_seqlens[s + 1] - cu_seqlens[s];
-            seqs.seq_id[r] = s;
-        }
-    } else {
-        S = B;
-        T = (long long)B * N;
-        seqs.varlen = 0;
-        seqs.N = N;
-    }
+    if (la_status st = build_seq_table(B, N, cu_seqlens, num_seqs, seqs, T, S); st != LA_OK)
+        return st;
     if (T >= (1ll << 31) || (long long)S * H * 2 >= (1ll << 31)) return LA_ERR_UNSUPPORTED;
     if (S == 0 || H == 0) return LA_OK;
 
@@ -241,6 +255,77 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
     if (beta == 64 && D == 128) return launch_simt<64, 128>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
     if (beta == 128 && D == 64) return launch_simt<128, 64>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
     return launch_simt<64, 64>(qf, kf, vf, of, state, state_in, H, rms, seqs, S, stream);
+}
+
+la_status la_chunk_state(const void *k, const void *v, int B, int H, int N, int D,
+                         const int32_t *cu_seqlens, int num_seqs, unsigned flags, float *state_out,
+                         void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (flags & ~(unsigned)LA_BF16) return LA_ERR_INVALID_ARG;
+    if (H < 1 || N < 0 || B < 1) return LA_ERR_INVALID_ARG;
+    if (N > 0 && (!k || !v)) return LA_ERR_INVALID_ARG;
+    if (!state_out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(state_out)) return LA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+    SeqTable seqs;
+    long long T = 0;
+    int S = 0;
+    if (la_status st = build_seq_table(B, N, cu_seqlens, num_seqs, seqs, T, S); st != LA_OK)
+        return st;
+    if (T >= (1ll << 31) || (long long)S * H * 2 >= (1ll << 31)) return LA_ERR_UNSUPPORTED;
+    if (S == 0) return LA_OK;
+    if (T == 0) {  // every sequence is empty: zero states
+        la::state_zero_kernel<<<(unsigned)(S * H), 256, 0, stream>>>(
+            reinterpret_cast<float4 *>(state_out), D * D / 4);
+        return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    }
+    if (flags & LA_BF16) {
+        la::ChunkStateParams p;
+        std::memset(&p, 0, sizeof p);
+        if (!make_map(&p.tmap_k, k, T, H, D, 128) || !make_map(&p.tmap_v, v, T, H, D, 128))
+            return LA_ERR_CUDA;
+        p.state = state_out;
+        p.H = H;
+        p.timeout_ns = kWaitLimitNs;
+        p.seqs = seqs;
+        auto launch = [&](auto kern, int smem, int threads, int nvs) -> la_status {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+                return LA_ERR_CUDA;
+            kern<<<(unsigned)(S * H * nvs), threads, smem, stream>>>(p);
+            return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+        };
+        if (D == 128)
+            return launch(la::chunk_state_tc_kernel<128>, la::ChunkCfg<128>::SMEM_BYTES,
+                          la::ChunkCfg<128>::THREADS, la::ChunkCfg<128>::NVS);
+        return launch(la::chunk_state_tc_kernel<64>, la::ChunkCfg<64>::SMEM_BYTES,
+                      la::ChunkCfg<64>::THREADS, la::ChunkCfg<64>::NVS);
+    }
+    const float *kf = static_cast<const float *>(k), *vf = static_cast<const float *>(v);
+    auto launch_simt_state = [&](auto kern, int Dv) -> la_status {
+        const int smem = (2 * 64 * Dv + Dv * Dv) * 4;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return LA_ERR_CUDA;
+        kern<<<(unsigned)(S * H), 256, smem, stream>>>(kf, vf, state_out, H, seqs);
+        return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    };
+    if (D == 128) return launch_simt_state(la::chunk_state_simt_kernel<128>, 128);
+    return launch_simt_state(la::chunk_state_simt_kernel<64>, 64);
+}
+
+la_status la_state_prefix(const float *gathered, int R, int rank, int S, int H, int D, float *out,
+                          void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (R < 1 || rank < 0 || rank > R || S < 0 || H < 1) return LA_ERR_INVALID_ARG;
+    if (!gathered || !out || !aligned16(gathered) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return LA_ERR_UNSUPPORTED;
+    if ((long long)S * H >= (1ll << 31)) return LA_ERR_UNSUPPORTED;
+    if (S == 0) return LA_OK;
+    const int n4 = D * D / 4;
+    la::state_prefix_kernel<<<(unsigned)(S * H), 256, 0, stream>>>(
+        reinterpret_cast<const float4 *>(gathered), reinterpret_cast<float4 *>(out), rank,
+        (size_t)S * H * n4, n4);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
 la_status la_decode_step(const void *q, const void *k, const void *v, float *state, void *o, int B,

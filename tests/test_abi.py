@@ -112,3 +112,27 @@ def test_decode_rejects(L, args, code):
 ])
 def test_state_out_rejects(L, args, code):
     assert L.la_state_out(*args, None) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((FAKE, FAKE, 1, 2, 8, 128, None, 0, 1 | 2, FAKE), api.LA_ERR_INVALID_ARG),   # flag not allowed
+    ((FAKE, FAKE, 1, 2, 8, 128, None, 0, 1, None), api.LA_ERR_INVALID_ARG),       # no output
+    ((None, FAKE, 1, 2, 8, 128, None, 0, 1, FAKE), api.LA_ERR_INVALID_ARG),       # no k
+    ((FAKE, FAKE, 1, 2, 8, 96, None, 0, 1, FAKE), api.LA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, 1, 0, 8, 128, None, 0, 1, FAKE), api.LA_ERR_INVALID_ARG),
+    ((FAKE, FAKE, 1, 2, 8, 128, None, 0, 1, FAKE + 8), api.LA_ERR_INVALID_ARG),   # misaligned
+])
+def test_chunk_state_rejects(L, args, code):
+    assert L.la_chunk_state(*args, None) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((FAKE, 0, 0, 1, 2, 128, FAKE), api.LA_ERR_INVALID_ARG),      # R < 1
+    ((FAKE, 2, 3, 1, 2, 128, FAKE), api.LA_ERR_INVALID_ARG),      # rank > R
+    ((FAKE, 2, -1, 1, 2, 128, FAKE), api.LA_ERR_INVALID_ARG),
+    ((None, 2, 1, 1, 2, 128, FAKE), api.LA_ERR_INVALID_ARG),
+    ((FAKE, 2, 1, 1, 2, 100, FAKE), api.LA_ERR_UNSUPPORTED),
+    ((FAKE, 2, 1, 0, 2, 128, FAKE), api.LA_OK),                   # nothing to do
+])
+def test_state_prefix_rejects(L, args, code):
+    assert L.la_state_prefix(*args, None) == code
