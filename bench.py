@@ -390,6 +390,7 @@ def run_ours(args):
         line["decode"], dctx = bench_decode(api, synth, torch, dev, stream, peak_bw, rank, world)
         line["concurrent"] = bench_concurrent(api, torch, stream, dctx, q, k, v, o, beta, world)
         del dctx
+        line["lasp_chunk_state"] = bench_chunk_state(api, torch, stream, k, v, peak_bw, world)
     if rank == 0 and not args.no_extras:
         line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
     if world > 1:
@@ -482,6 +483,29 @@ def bench_decode(api, synth, torch, dev, pstream, peak_bw, rank, world):
            "bytes_per_step": decode_bytes(B, H, D), "gpu_launches": steps,
            "status": api.status_string(status), "stream": "own stream (not the prefill stream)"}
     return res, (dstream, state, toks, outs)
+
+
+def bench_chunk_state(api, torch, stream, k, v, peak_bw, world, reps=5):
+    """Step 1 of LASP+ on the main workload's K and V: each sequence's K^T V alone.  It
+    reads 4 D bytes per token-head (K and V) and writes the fp32 states."""
+    H, D = k.shape[-2], k.shape[-1]
+    T = k.numel() // (H * D)
+    st = api.chunk_state(k, v, stream=stream)  # warm-up and allocation
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(reps):
+        api.chunk_state(k, v, state_out=st, stream=stream)
+        ev[i + 1].record(stream)
+    stream.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+    ms = statistics.median(per)
+    nbytes = 4 * D * T * H + st.numel() * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": "la::chunk_state_tc_kernel (the local state of a chunk in LASP+)",
+            "ms_median": ms, "bytes": nbytes, "gbs": gbs, "pct_hbm": 100.0 * gbs / peak_bw,
+            "launches": reps, "status": api.status_string(api.device_status(stream))}
 
 
 def bench_concurrent(api, torch, pstream, dctx, q, k, v, o, beta, world, n_prefill=2):
