@@ -143,6 +143,18 @@ la_status la_state_prefix(const float *gathered, int R, int rank, int S, int H, 
                           float *out, void *stream);
 
 /*
+ * la_selftest_wait -- exercise the device-side failure path.  Launches one small
+ * kernel whose single wait (on a barrier that nothing completes) gives up after
+ * limit_ns nanoseconds (clamped to 1 us .. 1 s), records LA_ERR_DEVICE_TIMEOUT in
+ * the device status word and returns; nothing else is in flight.  The next
+ * la_get_device_status on the stream reports LA_ERR_DEVICE_TIMEOUT and clears it;
+ * the context stays usable.  This is not part of the method (the pages describe no
+ * failure handling); it exists so that tests can check that bounded waits surface
+ * as errors instead of hangs.
+ */
+la_status la_selftest_wait(unsigned long long limit_ns, void *stream);
+
+/*
  * la_decode_step -- one token per sequence (length-1 path).
  *
  *   q, k, v   [B][H][D] the new token's projections (bf16 with LA_BF16, else fp32).

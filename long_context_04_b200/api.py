@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
     L.la_chunk_state.restype = i32
     L.la_state_prefix.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp]
     L.la_state_prefix.restype = i32
+    L.la_selftest_wait.argtypes = [ctypes.c_ulonglong, vp]
+    L.la_selftest_wait.restype = i32
     L.la_status_string.argtypes = [i32]
     L.la_status_string.restype = ctypes.c_char_p
     L.la_get_device_status.argtypes = [vp]
@@ -257,6 +259,12 @@ def state_prefix(gathered, rank: int, *, out=None, stream=None):
     rc = lib().la_state_prefix(_ptr(gathered), R, int(rank), S, H, D, _ptr(out), _stream_ptr(stream))
     _check("la_state_prefix", rc)
     return out
+
+
+def selftest_wait(limit_ns: int = 10_000_000, *, stream=None):
+    """Launch the self-test kernel whose one wait gives up after ``limit_ns``; the next
+    ``device_status`` reports LA_ERR_DEVICE_TIMEOUT."""
+    _check("la_selftest_wait", lib().la_selftest_wait(int(limit_ns), _stream_ptr(stream)))
 
 
 def device_status(stream=None) -> int:

@@ -16,6 +16,7 @@
 #include "prefill_simt.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -325,6 +326,14 @@ la_status la_state_prefix(const float *gathered, int R, int rank, int S, int H, 
     la::state_prefix_kernel<<<(unsigned)(S * H), 256, 0, stream>>>(
         reinterpret_cast<const float4 *>(gathered), reinterpret_cast<float4 *>(out), rank,
         (size_t)S * H * n4, n4);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_selftest_wait(unsigned long long limit_ns, void *stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (limit_ns < 1000ull) limit_ns = 1000ull;
+    if (limit_ns > kWaitLimitNs) limit_ns = kWaitLimitNs;
+    la::selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns);
     return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
