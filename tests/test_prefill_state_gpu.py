@@ -145,3 +145,32 @@ def test_long_paired_sequence_with_state_sampled_heads():
         assert api.device_status() == api.LA_OK
         assert oracle.max_rel_l2_per_head(o[:, heads], ref_o) <= 2e-2
         assert _state_err(st.cpu().numpy(), ref_s) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype,beta,D", [KERNELS[0], KERNELS[1], KERNELS[4]], ids=[IDS[0], IDS[1], IDS[4]])
+def test_mixed_batch_decode_and_prefill(dtype, beta, D):
+    """One launch over a packed mix of one-token sequences (decode) and longer chunks, each
+    continuing from its own state: the one-token rows equal the decode kernel's outputs,
+    every row and state equals the oracle's."""
+    H = 2
+    lens = [1, 1, 300, 1, 64, 0, 129]
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    S = len(lens)
+    q, k, v = synth.qkv(cu[-1], H, D, seed=36, dtype=dtype, device="cuda")
+    x = synth.initial_state(S, H, D, tokens=3000, seed=36, device="cuda")
+    st = x.clone()
+    o, _ = api.prefill(q, k, v, beta=beta, cu_seqlens=cu, initial_state=st, state_out=st)
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LA_OK
+    ref_o, ref_s = oracle.recurrent(q, k, v, cu, initial_state=x.cpu().numpy())
+    assert oracle.max_rel_l2_per_head(o, ref_o, cu) <= TOL[dtype]
+    assert _state_err(st.cpu().numpy(), ref_s) <= (1e-6 if dtype == torch.float32 else 1e-5)
+    # the one-token sequences through the decode kernel, from the same states
+    ones = [s for s in range(S) if lens[s] == 1]
+    rows = torch.as_tensor([cu[s] for s in ones], device="cuda")
+    dstate = x[ones].clone()
+    od = api.decode_step(q[rows].contiguous(), k[rows].contiguous(), v[rows].contiguous(), dstate)
+    torch.cuda.synchronize()
+    tol = 1e-5 if dtype == torch.float32 else 2e-2
+    assert oracle.rel_l2(o[rows], od) <= tol
+    assert oracle.rel_l2(st[ones], dstate) <= 1e-6
