@@ -391,7 +391,7 @@ def run_ours(args):
         line["concurrent"] = bench_concurrent(api, torch, stream, dctx, q, k, v, o, beta, world)
         del dctx
         line["lasp_chunk_state"] = bench_chunk_state(api, torch, stream, k, v, peak_bw, world)
-    if rank == 0 and not args.no_extras:
+    if rank == 0 and world == 1 and not args.no_extras:  # the host baseline is a 1-GPU figure
         line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
     if world > 1:
         import torch.distributed as dist
