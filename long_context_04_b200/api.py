@@ -92,13 +92,23 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else t.data_ptr()
 
 
+def _on_gpu(t: torch.Tensor) -> bool:
+    return t.is_cuda
+
+
 def _need(t: torch.Tensor, name: str, dtype=None):
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+    if not isinstance(t, torch.Tensor) or not _on_gpu(t):
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need_shape(t: torch.Tensor, name: str, shape):
+    # outputs are written through raw pointers: a wrong shape would be an out-of-bounds write
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
 def _flags_for(dtype) -> int:
@@ -147,11 +157,13 @@ def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
     if out is None:
         out = torch.empty_like(q)
     _need(out, "out", q.dtype)
+    _need_shape(out, "out", q.shape)
     st = state_out
     if return_state and st is None:
         st = torch.empty((S, H, D, D), dtype=torch.float32, device=q.device)
     if st is not None:
         _need(st, "state_out", torch.float32)
+        _need_shape(st, "state_out", (S, H, D, D))
         flags |= LA_WRITE_STATE
     ws = st
     if initial_state is not None:
@@ -163,7 +175,6 @@ def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
             ws = initial_state                       # read only
         elif st.data_ptr() != initial_state.data_ptr():
             _copy_state(initial_state, st, stream)   # the library's copy kernel; then in place
-    
     if rmsnorm:
         flags |= LA_OUT_RMSNORM
     cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
@@ -192,6 +203,8 @@ def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None)
         if t.shape != q.shape:
             raise ValueError("q, k, v must have one shape")
     _need(state, "state", torch.float32)
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, D]")
     B, H, D = q.shape
     if tuple(state.shape) != (B, H, D, D):
         raise ValueError("state must be [B, H, D, D]")
@@ -199,6 +212,7 @@ def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None)
     if out is None:
         out = torch.empty_like(q)
     _need(out, "out", q.dtype)
+    _need_shape(out, "out", q.shape)
     rc = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H, D, flags,
                               _stream_ptr(stream))
     _check("la_decode_step", rc)
@@ -209,9 +223,13 @@ def state_out(state_ws, state_dst, seq_to_slot=None, *, stream=None):
     """``state_dst[slot(s)] = state_ws[s]`` (slot = ``seq_to_slot[s]``, a CUDA int32 tensor)."""
     _need(state_ws, "state_ws", torch.float32)
     _need(state_dst, "state_dst", torch.float32)
+    if state_ws.dim() != 4 or state_dst.dim() != 4:
+        raise ValueError("state_ws and state_dst must be [*, H, D, D]")
     S, H, D, _ = state_ws.shape
+    _need_shape(state_dst, "state_dst", (state_dst.shape[0], H, D, D))
     if seq_to_slot is not None:
         _need(seq_to_slot, "seq_to_slot", torch.int32)
+        _need_shape(seq_to_slot, "seq_to_slot", (S,))
     rc = lib().la_state_out(_ptr(state_ws), _ptr(state_dst), S, H, D, _ptr(seq_to_slot),
                             state_dst.shape[0], _stream_ptr(stream))
     _check("la_state_out", rc)
@@ -241,6 +259,7 @@ def chunk_state(k, v, *, cu_seqlens=None, state_out=None, stream=None):
     if state_out is None:
         state_out = torch.empty((S, H, D, D), dtype=torch.float32, device=k.device)
     _need(state_out, "state_out", torch.float32)
+    _need_shape(state_out, "state_out", (S, H, D, D))
     cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
     rc = lib().la_chunk_state(_ptr(k), _ptr(v), B, H, N, D, cu_ptr, 0 if cu is None else len(cu) - 1,
                               flags, _ptr(state_out), _stream_ptr(stream))
@@ -252,10 +271,13 @@ def state_prefix(gathered, rank: int, *, out=None, stream=None):
     """``out = sum_{r < rank} gathered[r]`` for gathered ``[R, S, H, D, D]`` fp32 (the
     chunk states of all ranks): the initial state of chunk ``rank`` in LASP+."""
     _need(gathered, "gathered", torch.float32)
+    if gathered.dim() != 5:
+        raise ValueError("gathered must be [R, S, H, D, D]")
     R, S, H, D, _ = gathered.shape
     if out is None:
         out = torch.empty((S, H, D, D), dtype=torch.float32, device=gathered.device)
     _need(out, "out", torch.float32)
+    _need_shape(out, "out", (S, H, D, D))
     rc = lib().la_state_prefix(_ptr(gathered), R, int(rank), S, H, D, _ptr(out), _stream_ptr(stream))
     _check("la_state_prefix", rc)
     return out
