@@ -72,10 +72,11 @@ def test_state_out_out_of_range_slot_is_reported():
 def test_config5_decode_from_prefill_state():
     """B=256, H=64, D=128: state from seeded N=4096 prefills (8 chunks of 32 sequences,
     handed over with la_state_out), then 64 decode steps.  Checks: step 1 for every (b, h)
-    from the exact GPU input state; 4 sampled (b, h) from scratch in fp64 over all 64 steps."""
+    from the exact GPU input state; 64 sampled (b, h) from scratch in fp64 over all 64 steps."""
     B, H, D, N, steps, chunk = 256, 64, 128, 4096, 64, 32
     state = torch.empty(B, H, D, D, device="cuda")
-    sample = [(0, 0), (77, 13), (130, 40), (255, 63)]
+    # 64 pairs with distinct b (37 is odd, so i -> 37 i + 5 mod 256 is one-to-one), corners included
+    sample = [(0, 0), (255, 63)] + [((37 * i + 5) % 256, (29 * i + 3) % 64) for i in range(62)]
     kept = {}
     for c in range(B // chunk):
         q, k, v = synth.qkv(chunk * N, H, D, seed=100 + c, dtype=torch.bfloat16, device="cuda")
