@@ -137,7 +137,7 @@ def test_config2_layer_prefill(beta):
 
 
 def test_config3_long_context():
-    """B=1, H=64, N=131072, D=128, beta=128: heads {0, 37} + 16 sampled final states."""
+    """B=1, H=64, N=131072, D=128, beta=128: heads {0, 37} in full + every head's final state."""
     T, H, D = 131072, 64, 128
     q, k, v = synth.qkv(T, H, D, seed=0, dtype=torch.bfloat16, device="cuda")
     o, st = api.prefill(q, k, v, beta=128, return_state=True)
@@ -147,9 +147,10 @@ def test_config3_long_context():
     o_ref, st_ref = oracle.recurrent(q[:, heads], k[:, heads], v[:, heads])
     assert oracle.max_rel_l2_per_head(o[:, heads], o_ref) <= 2e-2
     assert _state_err(st[:, heads].cpu().double().numpy(), st_ref) <= 2e-2
-    sample = list(range(0, 64, 4))
-    st_ref2 = oracle.final_state(k[:, sample], v[:, sample])
-    assert _state_err(st[:, sample].cpu().double().numpy(), st_ref2) <= 2e-2
+    for h0 in range(0, H, 16):  # 16 heads at a time keeps the fp64 copies of K, V near 4 GB
+        hs = list(range(h0, h0 + 16))
+        st_ref2 = oracle.final_state(k[:, hs], v[:, hs])
+        assert _state_err(st[:, hs].cpu().double().numpy(), st_ref2) <= 2e-2
     assert bool(torch.isfinite(o).all())
 
 
