@@ -40,6 +40,48 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def _declared_signatures():
+    """name -> parameter kinds ("ptr", "i32", "u32", "u64") from the header declarations."""
+    sigs = {}
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", fn)).read(), flags=re.S)
+        for name, params in re.findall(r"\b(la_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text):
+            kinds = []
+            for prm in (x.strip() for x in params.split(",")):
+                if prm in ("", "void"):
+                    continue
+                if "*" in prm:
+                    kinds.append("ptr")
+                elif prm.startswith("unsigned long long"):
+                    kinds.append("u64")
+                elif prm.startswith("unsigned"):
+                    kinds.append("u32")
+                elif prm.startswith(("int ", "la_status ")):
+                    kinds.append("i32")
+                else:
+                    raise AssertionError(f"{name}: unclassified parameter {prm!r}")
+            sigs[name] = kinds
+    return sigs
+
+
+def _ctypes_kind(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    return {ctypes.c_int: "i32", ctypes.c_uint: "u32", ctypes.c_ulonglong: "u64"}[t]
+
+
+def test_binding_argtypes_match_the_header(L):
+    """Every declared entry point is called with the header's parameter list: a drifted
+    argtypes entry would pass arguments in the wrong registers without any error."""
+    sigs = _declared_signatures()
+    assert set(sigs) == set(_declared_functions())
+    for name, kinds in sigs.items():
+        got = [_ctypes_kind(t) for t in (getattr(L, name).argtypes or [])]
+        assert got == kinds, (name, got, kinds)
+
+
 def test_status_strings(L):
     for code, text in [(0, "LA_OK"), (1, "LA_ERR_INVALID_ARG"), (2, "LA_ERR_UNSUPPORTED"),
                        (3, "LA_ERR_CUDA"), (4, "LA_ERR_DEVICE_TIMEOUT"),
