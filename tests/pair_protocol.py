@@ -14,7 +14,8 @@ Asynchronous work is a pool of pending events that fire in random order, interle
 random with the agents' steps: each TMA tile landing (its transaction bytes on its
 barrier), each MMA's completion (in issue order per issuing thread, the two threads
 independent), each commit's arrival on each CTA's barrier, and each arrival that a
-CTA 1 thread sends to a CTA 0 barrier.
+CTA 1 thread sends to a CTA 0 barrier.  Every schedule draws a speed for each agent and
+each kind of event, so that some schedules starve one role for long stretches.
 
 Every schedule is checked for:
   * the parity-wait rules: a wait (or the producer's non-blocking test) on phase n of a
@@ -469,6 +470,16 @@ class PairModel:
                 other[1] = True
                 yield STEP
 
+    def agents(self):
+        """name -> generator, one per role of the kernel."""
+        agents = {"producer0": self.producer(0), "producer1": self.producer(1),
+                  "A": self.issuer_a(), "B": self.issuer_b()}
+        for c in (0, 1):
+            for w in range(WARPS):
+                agents[f"P{c}.{w}"] = self.group_p(c, w)
+                agents[f"O{c}.{w}"] = self.group_o(c, w)
+        return agents
+
     # ------------------------------------------------------------------ scheduler
     def _events(self):
         evs = list(self.inflight)
@@ -516,13 +527,13 @@ class PairModel:
         the first violation."""
         rng = random.Random(seed)
         bias = rng.uniform(0.05, 0.95)      # how eagerly asynchronous work completes
-        agents = {"producer0": self.producer(0), "producer1": self.producer(1),
-                  "A": self.issuer_a(), "B": self.issuer_b()}
-        for c in (0, 1):
-            for w in range(WARPS):
-                agents[f"P{c}.{w}"] = self.group_p(c, w)
-                agents[f"O{c}.{w}"] = self.group_o(c, w)
+        agents = self.agents()
         state = {name: ("ready",) for name in agents}
+        # Each agent and each kind of asynchronous event gets a speed for this schedule, so
+        # that some schedules starve one role (a slow warp, late TMA tiles, a slow issuer).
+        speeds = (0.02, 0.2, 1.0, 1.0, 5.0)
+        w_agent = {name: rng.choice(speeds) for name in agents}
+        w_event = {kind: rng.choice(speeds) for kind in ("tma", "arrive", "mma", "commit")}
         for _ in range(max_steps):
             live = [n for n, st in state.items() if st[0] != "done"]
             runnable = [n for n in live if self._runnable(state[n])]
@@ -534,9 +545,9 @@ class PairModel:
                     f"{n} waits on phase {state[n][2]} of {state[n][1].name}" if state[n][0] == "wait"
                     else f"{n} polls" for n in live))
             if events and (not runnable or rng.random() < bias):
-                self._fire(rng.choice(events))
+                self._fire(rng.choices(events, weights=[w_event[e.kind] for e in events])[0])
             else:
-                name = rng.choice(runnable)
+                name = rng.choices(runnable, weights=[w_agent[n] for n in runnable])[0]
                 try:
                     instr = next(agents[name])
                 except StopIteration:
