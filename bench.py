@@ -10,8 +10,9 @@ with Q/K/V/O (8.6 GB) resident in HBM.  The inputs are far larger than the
 tokens/s over all ranks; the JSON line also carries the tensor-core view
 (TFLOP/s, % of bf16 peak), the decode step (B=256, H=64, D=128, fp32 state of a
 seeded N=4096 prefill; tokens/s and % of HBM bandwidth), the roofline of the
-prefill kernel, the end-to-end number through the C ABI with host buffers, and
-the fp64 oracle timed on the host cores as a CPU baseline.
+prefill kernel, the end-to-end number through the C ABI with host buffers, a
+sweep of the sequence length at a fixed token count, and the fp64 oracle timed on
+the host cores as a CPU baseline.
 
 Multi-GPU (torchrun): every rank runs its own copy of the workload on its own
 GPU (independent problems, no data-path collective: weak scaling); the timed
@@ -391,6 +392,11 @@ def run_ours(args):
         line["concurrent"] = bench_concurrent(api, torch, stream, dctx, q, k, v, o, beta, world)
         del dctx
         line["lasp_chunk_state"] = bench_chunk_state(api, torch, stream, k, v, peak_bw, world)
+        if world == 1:  # rank-local extra: no collective, so a failure cannot strand other ranks
+            try:
+                line["length_sweep"] = bench_length_sweep(api, torch, stream, q, k, v, o, beta, peak_bw)
+            except Exception as e:  # an extra that fails must not cost the main line
+                line["length_sweep"] = {"error": repr(e)}
     if rank == 0 and world == 1 and not args.no_extras:  # the host baseline is a 1-GPU figure
         line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
     if world > 1:
@@ -483,6 +489,48 @@ def bench_decode(api, synth, torch, dev, pstream, peak_bw, rank, world):
            "bytes_per_step": decode_bytes(B, H, D), "gpu_launches": steps,
            "status": api.status_string(status), "stream": "own stream (not the prefill stream)"}
     return res, (dstream, state, toks, outs)
+
+
+SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072)
+
+
+def sweep_row(N, T, H, D, beta, ms, peak_bw, status):
+    """One point of the length sweep: B = T / N sequences of N tokens in one launch."""
+    s = ms / 1e3
+    return {"N": N, "B": T // N, "ms_per_launch": ms, "tokens_per_s": T / s,
+            "tflops_tiled": tiled_flops_per_token_head(D, beta) * T * H / s / 1e12,
+            "hbm_frac": prefill_bytes(T, H, D) / s / 1e9 / peak_bw, "status": status}
+
+
+def bench_length_sweep(api, torch, stream, q, k, v, o, beta, peak_bw, reps=20, warm=3):
+    """Prefill speed against sequence length at a fixed token count per launch.
+
+    The main workload's Q/K/V/O (T tokens x H heads) are viewed as B = T / N sequences of N
+    tokens, N = 1K .. 128K, so every launch reads and writes the same bytes.  Attention that
+    is linear in N keeps the time per launch independent of N; the pages claim a constant
+    speed over 1K-64K tokens (measured against FlashAttention-2 on other GPUs)."""
+    H, D = q.shape[-2], q.shape[-1]
+    T = q.numel() // (H * D)
+    rows = []
+    for N in SWEEP_N:
+        if N > T or T % N:
+            continue
+        B = T // N
+        qv, kv_, vv, ov = (x.reshape(B, N, H, D) for x in (q, k, v, o))
+        for _ in range(warm):
+            api.prefill(qv, kv_, vv, beta=beta, out=ov, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            api.prefill(qv, kv_, vv, beta=beta, out=ov, stream=stream)
+        e1.record(stream)
+        stream.synchronize()
+        status = api.status_string(api.device_status(stream))
+        rows.append(sweep_row(N, T, H, D, beta, e0.elapsed_time(e1) / reps, peak_bw, status))
+    return {"what": "prefill at a fixed T x H per launch, as B = T / N sequences of N tokens",
+            "tokens_per_launch": T, "heads": H, "head_dim": D, "beta": beta,
+            "launches_per_point": reps, "rows": rows}
 
 
 def bench_chunk_state(api, torch, stream, k, v, peak_bw, world, reps=5):

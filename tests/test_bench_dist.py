@@ -67,3 +67,68 @@ def test_single_process_helpers_are_identities():
     assert bench.tiled_flops_per_token_head(128, 128) == 131072
     assert bench.prefill_bytes(131072, 64, 128) == 8589934592
     assert bench.decode_bytes(256, 64, 128) == 2164260864
+
+
+class _Event:
+    clock = 0.0
+
+    def __init__(self, enable_timing=True):
+        self.t = None
+
+    def record(self, stream=None):
+        _Event.clock += 1.0
+        self.t = _Event.clock
+
+    def elapsed_time(self, other):
+        return (other.t - self.t) * 1000.0
+
+
+class _FakeTorch:
+    class cuda:
+        Event = _Event
+
+        @staticmethod
+        def synchronize():
+            pass
+
+
+class _FakeStream:
+    def synchronize(self):
+        pass
+
+
+class _FakeApi:
+    def __init__(self):
+        self.shapes = []
+
+    def prefill(self, q, k, v, beta, out, stream):
+        assert q.shape == k.shape == v.shape == out.shape and out.data_ptr() == self.o_ptr
+        self.shapes.append(tuple(q.shape))
+
+    def device_status(self, stream=None):
+        return 0
+
+    def status_string(self, status):
+        return "LA_OK"
+
+
+def test_length_sweep_control_flow():
+    """The sweep's host logic with stand-ins for CUDA events, the stream and the library:
+    views of the one workload as B = T / N sequences, warm-up + timed launches per N, and
+    one row per N that divides T."""
+    import torch
+
+    import bench
+    T, H, D = 4096, 2, 8
+    q, k, v, o = (torch.zeros(1, T, H, D) for _ in range(4))
+    api = _FakeApi()
+    api.o_ptr = o.data_ptr()
+    res = bench.bench_length_sweep(api, _FakeTorch, _FakeStream(), q, k, v, o, 128, 6544.0, reps=4, warm=2)
+    assert [r["N"] for r in res["rows"]] == [1024, 2048, 4096]
+    assert [r["B"] for r in res["rows"]] == [4, 2, 1]
+    assert api.shapes.count((4, 1024, H, D)) == 6 and api.shapes.count((1, 4096, H, D)) == 6
+    r = res["rows"][0]
+    assert r["ms_per_launch"] == pytest.approx(1000.0 / 4)    # one fake second over 4 launches
+    assert r["tokens_per_s"] == pytest.approx(T / 0.25)
+    assert r["hbm_frac"] == pytest.approx(8 * T * H * D / 0.25 / 1e9 / 6544.0)
+    assert r["status"] == "LA_OK" and res["tokens_per_launch"] == T
