@@ -397,6 +397,10 @@ def run_ours(args):
                 line["length_sweep"] = bench_length_sweep(api, torch, stream, q, k, v, o, beta, peak_bw)
             except Exception as e:  # an extra that fails must not cost the main line
                 line["length_sweep"] = {"error": repr(e)}
+            try:
+                line["prefill_options"] = bench_prefill_options(api, torch, stream, q, k, v, o, peak_bw)
+            except Exception as e:
+                line["prefill_options"] = {"error": repr(e)}
     if rank == 0 and world == 1 and not args.no_extras:  # the host baseline is a 1-GPU figure
         line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
     if world > 1:
@@ -531,6 +535,36 @@ def bench_length_sweep(api, torch, stream, q, k, v, o, beta, peak_bw, reps=20, w
     return {"what": "prefill at a fixed T x H per launch, as B = T / N sequences of N tokens",
             "tokens_per_launch": T, "heads": H, "head_dim": D, "beta": beta,
             "launches_per_point": reps, "rows": rows}
+
+
+def bench_prefill_options(api, torch, stream, q, k, v, o, peak_bw, reps=10, warm=3):
+    """The main workload through the other options of la_prefill, each timed alone: the fused
+    output RMSNorm, beta = 64 (the unpaired tcgen05 kernel) and a start from an initial
+    state (read only; the inter-block term of block 0 is then computed too)."""
+    H, D = q.shape[-2], q.shape[-1]
+    T = q.numel() // (H * D)
+    S = q.shape[0] if q.dim() == 4 else 1
+    X = torch.zeros((S, H, D, D), dtype=torch.float32, device=q.device)
+    cases = {"rmsnorm": dict(beta=128, rmsnorm=True),
+             "beta64": dict(beta=64),
+             "initial_state": dict(beta=128, initial_state=X)}
+    res = {}
+    for name, kw in cases.items():
+        for _ in range(warm):
+            api.prefill(q, k, v, out=o, stream=stream, **kw)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            api.prefill(q, k, v, out=o, stream=stream, **kw)
+        e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = {"ms_per_launch": ms, "tokens_per_s": T / (ms / 1e3),
+                     "hbm_frac": prefill_bytes(T, H, D) / (ms / 1e3) / 1e9 / peak_bw,
+                     "status": api.status_string(api.device_status(stream))}
+    res["launches_per_option"] = reps
+    return res
 
 
 def bench_chunk_state(api, torch, stream, k, v, peak_bw, world, reps=5):

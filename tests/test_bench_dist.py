@@ -84,6 +84,10 @@ class _Event:
 
 
 class _FakeTorch:
+    import torch as _torch
+    zeros = staticmethod(_torch.zeros)
+    float32 = _torch.float32
+
     class cuda:
         Event = _Event
 
@@ -100,10 +104,15 @@ class _FakeStream:
 class _FakeApi:
     def __init__(self):
         self.shapes = []
+        self.options = []
 
-    def prefill(self, q, k, v, beta, out, stream):
+    def prefill(self, q, k, v, beta=128, out=None, stream=None, rmsnorm=False, initial_state=None):
         assert q.shape == k.shape == v.shape == out.shape and out.data_ptr() == self.o_ptr
+        assert beta in (64, 128)
+        if initial_state is not None:
+            assert tuple(initial_state.shape) == (q.shape[0], q.shape[2], q.shape[3], q.shape[3])
         self.shapes.append(tuple(q.shape))
+        self.options.append((beta, rmsnorm, initial_state is not None))
 
     def device_status(self, stream=None):
         return 0
@@ -132,3 +141,19 @@ def test_length_sweep_control_flow():
     assert r["tokens_per_s"] == pytest.approx(T / 0.25)
     assert r["hbm_frac"] == pytest.approx(8 * T * H * D / 0.25 / 1e9 / 6544.0)
     assert r["status"] == "LA_OK" and res["tokens_per_launch"] == T
+
+
+def test_prefill_options_control_flow():
+    import torch
+
+    import bench
+    T, H, D = 2048, 2, 8
+    q, k, v, o = (torch.zeros(1, T, H, D) for _ in range(4))
+    api = _FakeApi()
+    api.o_ptr = o.data_ptr()
+    res = bench.bench_prefill_options(api, _FakeTorch, _FakeStream(), q, k, v, o, 6544.0, reps=3, warm=1)
+    assert set(res) == {"rmsnorm", "beta64", "initial_state", "launches_per_option"}
+    assert api.options.count((128, True, False)) == 4
+    assert api.options.count((64, False, False)) == 4
+    assert api.options.count((128, False, True)) == 4
+    assert res["beta64"]["ms_per_launch"] == pytest.approx(1000.0 / 3)
