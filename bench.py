@@ -371,6 +371,8 @@ def run_ours(args):
                     "bf16_peak_tflops": peak_tf,
                     "roofline_ceiling_tflops": min(peak_tf, flops / alg_bytes * peak_bw / 1e3),
                     "avg_launch_ms": avg_launch_s * 1e3,
+                    "launch_ms_min_median_max": [min(launch_ms), statistics.median(launch_ms),
+                                                 max(launch_ms)],
                     "flops_per_token_head": tiled_flops_per_token_head(D, beta)}
 
     line = {
