@@ -83,7 +83,10 @@ enum {
  *             (data packing: sequences concatenated along the token axis, CSDN
  *             digest section 3.2).  The state is reset at every boundary;
  *             zero-length sequences are allowed.  NULL = B equal sequences.
- *             The array is read during the call only.
+ *             The array is read during the call only.  It is a host array on
+ *             purpose, not a device one: the library validates it before the
+ *             launch and passes the (longest-first) sequence table in the kernel
+ *             parameters, so a call needs no device scratch and no synchronisation.
  *   num_seqs  entries of cu_seqlens minus one (1 .. LA_MAX_VARLEN_SEQS); ignored
  *             when cu_seqlens is NULL.
  *   flags     LA_BF16 or LA_FP32, optionally | LA_OUT_RMSNORM | LA_WRITE_STATE
@@ -173,6 +176,8 @@ la_status la_decode_step(const void *q, const void *k, const void *v, float *sta
  *
  *   state_ws    [S][H][D][D] fp32 source (as written by la_prefill).
  *   state_dst   [num_slots][H][D][D] fp32 destination (the decode batch state).
+ *   num_slots   rows of state_dst.  Given explicitly, so that a slot index read on
+ *               the device can be range-checked there.
  *   seq_to_slot DEVICE array of S int32 slot indices, or NULL (identity; then
  *               S <= num_slots is required).  A slot outside [0, num_slots) is
  *               skipped on the device and reported as LA_ERR_DEVICE_RANGE by
@@ -189,7 +194,10 @@ const char *la_status_string(la_status status);
  * la_get_device_status -- synchronise `stream`, then return and clear the
  * current device's status word: LA_OK, LA_ERR_DEVICE_TIMEOUT or
  * LA_ERR_DEVICE_RANGE (the first recorded), or LA_ERR_CUDA if the stream
- * reports an error.  The word is shared by every call on the device.
+ * reports an error.  The word is per device, not per stream: it is shared by
+ * every call on the device, so with prefill and decode on two streams a fault
+ * recorded by either kernel is reported to (and cleared by) whichever
+ * la_get_device_status call on that device comes first.
  */
 la_status la_get_device_status(void *stream);
 

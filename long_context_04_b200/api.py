@@ -96,13 +96,45 @@ def _on_gpu(t: torch.Tensor) -> bool:
     return t.is_cuda
 
 
-def _need(t: torch.Tensor, name: str, dtype=None):
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
     if not isinstance(t, torch.Tensor) or not _on_gpu(t):
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    # the library launches on the current device: every pointer of a call must live there
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's tensors on {device}")
+
+
+class _on_device:
+    """Make ``dev`` the current CUDA device for one library call (the library launches,
+    builds tensor maps and reads the status word on the current device), and check
+    that an explicit stream belongs to it."""
+
+    def __init__(self, dev, stream=None):
+        self.dev = dev
+        if stream is not None and getattr(stream, "device", dev) != dev:
+            raise ValueError(f"stream is on {stream.device}, the call's tensors on {dev}")
+
+    def __enter__(self):
+        self.ctx = torch.cuda.device(self.dev) if self.dev.type == "cuda" else None
+        if self.ctx is not None:
+            self.ctx.__enter__()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ctx is not None:
+            self.ctx.__exit__(*exc)
+        return False
+
+
+def _overlap(a: torch.Tensor, b: torch.Tensor) -> bool:
+    """Whether the byte ranges of two tensors intersect."""
+    a0, b0 = a.data_ptr(), b.data_ptr()
+    a1, b1 = a0 + a.numel() * a.element_size(), b0 + b.numel() * b.element_size()
+    return a0 < b1 and b0 < a1
 
 
 def _need_shape(t: torch.Tensor, name: str, shape):
@@ -132,11 +164,13 @@ def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
     ``initial_state`` (``[S, H, D, D]`` fp32): each sequence continues from it
     (chunked prefill, resume).  The final state then is ``initial + K^T V``; it
     is written over ``initial_state`` itself when ``state_out`` is that tensor,
-    otherwise ``initial_state`` is left as it is.
+    otherwise ``initial_state`` is left as it is (``state_out`` must then not
+    overlap it).
     """
     _need(q, "q")
+    dev = q.device
     for t, n in ((k, "k"), (v, "v")):
-        _need(t, n, q.dtype)
+        _need(t, n, q.dtype, dev)
         if t.shape != q.shape:
             raise ValueError("q, k, v must have one shape")
     flags = _flags_for(q.dtype)
@@ -156,30 +190,39 @@ def prefill(q, k, v, *, beta: int = 128, cu_seqlens=None, rmsnorm: bool = False,
         cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", q.dtype)
+    _need(out, "out", q.dtype, dev)
     _need_shape(out, "out", q.shape)
     st = state_out
     if return_state and st is None:
-        st = torch.empty((S, H, D, D), dtype=torch.float32, device=q.device)
+        st = torch.empty((S, H, D, D), dtype=torch.float32, device=dev)
     if st is not None:
-        _need(st, "state_out", torch.float32)
+        _need(st, "state_out", torch.float32, dev)
         _need_shape(st, "state_out", (S, H, D, D))
         flags |= LA_WRITE_STATE
     ws = st
+    copy_in = False
     if initial_state is not None:
-        _need(initial_state, "initial_state", torch.float32)
+        _need(initial_state, "initial_state", torch.float32, dev)
         if tuple(initial_state.shape) != (S, H, D, D):
             raise ValueError("initial_state must be [S, H, D, D]")
         flags |= LA_READ_STATE
         if st is None:
             ws = initial_state                       # read only
         elif st.data_ptr() != initial_state.data_ptr():
-            _copy_state(initial_state, st, stream)   # the library's copy kernel; then in place
+            # copied into state_out by the library, then updated there in place; a partial
+            # overlap would overwrite initial state values before they are read
+            if _overlap(st, initial_state):
+                raise ValueError("state_out and initial_state overlap without coinciding")
+            copy_in = True
     if rmsnorm:
         flags |= LA_OUT_RMSNORM
     cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
-    rc = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, D, beta, cu_ptr,
-                          0 if cu is None else len(cu) - 1, flags, _ptr(ws), _stream_ptr(stream))
+    with _on_device(dev, stream):
+        if copy_in:
+            _copy_state(initial_state, st, stream)   # the library's copy kernel
+        rc = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, D, beta, cu_ptr,
+                              0 if cu is None else len(cu) - 1, flags, _ptr(ws),
+                              _stream_ptr(stream))
     _check("la_prefill", rc)
     return (out, st) if (return_state or state_out is not None) else out
 
@@ -198,11 +241,12 @@ def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None)
     ``q, k, v``: ``[B, H, D]``; ``state``: ``[B, H, D, D]`` fp32.
     """
     _need(q, "q")
+    dev = q.device
     for t, n in ((k, "k"), (v, "v")):
-        _need(t, n, q.dtype)
+        _need(t, n, q.dtype, dev)
         if t.shape != q.shape:
             raise ValueError("q, k, v must have one shape")
-    _need(state, "state", torch.float32)
+    _need(state, "state", torch.float32, dev)
     if q.dim() != 3:
         raise ValueError("q must be [B, H, D]")
     B, H, D = q.shape
@@ -211,10 +255,11 @@ def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None)
     flags = _flags_for(q.dtype) | (LA_OUT_RMSNORM if rmsnorm else 0)
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", q.dtype)
+    _need(out, "out", q.dtype, dev)
     _need_shape(out, "out", q.shape)
-    rc = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H, D, flags,
-                              _stream_ptr(stream))
+    with _on_device(dev, stream):
+        rc = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), B, H, D,
+                                  flags, _stream_ptr(stream))
     _check("la_decode_step", rc)
     return out
 
@@ -222,16 +267,20 @@ def decode_step(q, k, v, state, *, rmsnorm: bool = False, out=None, stream=None)
 def state_out(state_ws, state_dst, seq_to_slot=None, *, stream=None):
     """``state_dst[slot(s)] = state_ws[s]`` (slot = ``seq_to_slot[s]``, a CUDA int32 tensor)."""
     _need(state_ws, "state_ws", torch.float32)
-    _need(state_dst, "state_dst", torch.float32)
+    dev = state_ws.device
+    _need(state_dst, "state_dst", torch.float32, dev)
     if state_ws.dim() != 4 or state_dst.dim() != 4:
         raise ValueError("state_ws and state_dst must be [*, H, D, D]")
     S, H, D, _ = state_ws.shape
     _need_shape(state_dst, "state_dst", (state_dst.shape[0], H, D, D))
+    if _overlap(state_ws, state_dst):
+        raise ValueError("state_ws and state_dst must not overlap")
     if seq_to_slot is not None:
-        _need(seq_to_slot, "seq_to_slot", torch.int32)
+        _need(seq_to_slot, "seq_to_slot", torch.int32, dev)
         _need_shape(seq_to_slot, "seq_to_slot", (S,))
-    rc = lib().la_state_out(_ptr(state_ws), _ptr(state_dst), S, H, D, _ptr(seq_to_slot),
-                            state_dst.shape[0], _stream_ptr(stream))
+    with _on_device(dev, stream):
+        rc = lib().la_state_out(_ptr(state_ws), _ptr(state_dst), S, H, D, _ptr(seq_to_slot),
+                                state_dst.shape[0], _stream_ptr(stream))
     _check("la_state_out", rc)
     return state_dst
 
@@ -240,7 +289,8 @@ def chunk_state(k, v, *, cu_seqlens=None, state_out=None, stream=None):
     """Each sequence's K^T V alone (no output): ``[S, H, D, D]`` fp32.  The local state
     of a chunk in LASP+ sequence parallelism."""
     _need(k, "k")
-    _need(v, "v", k.dtype)
+    dev = k.device
+    _need(v, "v", k.dtype, dev)
     if v.shape != k.shape:
         raise ValueError("k and v must have one shape")
     flags = _flags_for(k.dtype)
@@ -257,12 +307,14 @@ def chunk_state(k, v, *, cu_seqlens=None, state_out=None, stream=None):
         raise ValueError("k must be [B, N, H, D] or [T, H, D]")
     cu = None if cu_seqlens is None else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
     if state_out is None:
-        state_out = torch.empty((S, H, D, D), dtype=torch.float32, device=k.device)
-    _need(state_out, "state_out", torch.float32)
+        state_out = torch.empty((S, H, D, D), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", torch.float32, dev)
     _need_shape(state_out, "state_out", (S, H, D, D))
     cu_ptr = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
-    rc = lib().la_chunk_state(_ptr(k), _ptr(v), B, H, N, D, cu_ptr, 0 if cu is None else len(cu) - 1,
-                              flags, _ptr(state_out), _stream_ptr(stream))
+    with _on_device(dev, stream):
+        rc = lib().la_chunk_state(_ptr(k), _ptr(v), B, H, N, D, cu_ptr,
+                                  0 if cu is None else len(cu) - 1, flags, _ptr(state_out),
+                                  _stream_ptr(stream))
     _check("la_chunk_state", rc)
     return state_out
 
@@ -271,14 +323,19 @@ def state_prefix(gathered, rank: int, *, out=None, stream=None):
     """``out = sum_{r < rank} gathered[r]`` for gathered ``[R, S, H, D, D]`` fp32 (the
     chunk states of all ranks): the initial state of chunk ``rank`` in LASP+."""
     _need(gathered, "gathered", torch.float32)
+    dev = gathered.device
     if gathered.dim() != 5:
         raise ValueError("gathered must be [R, S, H, D, D]")
     R, S, H, D, _ = gathered.shape
     if out is None:
-        out = torch.empty((S, H, D, D), dtype=torch.float32, device=gathered.device)
-    _need(out, "out", torch.float32)
+        out = torch.empty((S, H, D, D), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
     _need_shape(out, "out", (S, H, D, D))
-    rc = lib().la_state_prefix(_ptr(gathered), R, int(rank), S, H, D, _ptr(out), _stream_ptr(stream))
+    if _overlap(gathered, out):
+        raise ValueError("out must not overlap gathered")
+    with _on_device(dev, stream):
+        rc = lib().la_state_prefix(_ptr(gathered), R, int(rank), S, H, D, _ptr(out),
+                                   _stream_ptr(stream))
     _check("la_state_prefix", rc)
     return out
 

@@ -30,6 +30,7 @@ Every array is float64 ``[T, H, D]``; ``cu_seqlens`` has S+1 entries.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import numpy as np
@@ -180,8 +181,19 @@ def final_state(k, v, cu_seqlens=None) -> np.ndarray:
 
 
 def rel_l2(x, ref) -> float:
-    """||x - ref||_2 / ||ref||_2 in fp64 (0 when both are zero)."""
+    """||x - ref||_2 / ||ref||_2 in fp64: the error metric of the parity tests.
+
+    Returns 0 when both are zero, and inf when ``x`` holds a NaN or an infinity or
+    when ``ref`` is zero and ``x`` is not, so that a non-finite or spurious output
+    can never pass a tolerance.  The shapes must agree and ``ref`` must be finite.
+    """
     x, ref = _f64(x), _f64(ref)
+    if x.shape != ref.shape:
+        raise ValueError(f"shapes differ: {x.shape} vs {ref.shape}")
+    if not np.isfinite(ref).all():
+        raise ValueError("the reference holds a non-finite value")
+    if not np.isfinite(x).all():
+        return float("inf")
     den = float(np.linalg.norm(ref.ravel()))
     num = float(np.linalg.norm((x - ref).ravel()))
     if den == 0.0:
@@ -189,16 +201,46 @@ def rel_l2(x, ref) -> float:
     return num / den
 
 
+def _worse(worst: float, e: float) -> float:
+    # a NaN error counts as infinitely bad (Python's max() would drop it)
+    if math.isnan(e):
+        return float("inf")
+    return e if e > worst else worst
+
+
 def max_rel_l2_per_head(x, ref, cu_seqlens=None) -> float:
-    """Maximum over (sequence, head) of the relative L2 error on [T, H, D] arrays."""
+    """Maximum over (sequence, head) of the relative L2 error on ``[T, H, D]`` arrays:
+    ``max_{s,h} ||x[a_s:b_s, h] - ref[a_s:b_s, h]|| / ||ref[a_s:b_s, h]||`` with
+    ``[a_s, b_s)`` the rows of sequence s (all T rows when ``cu_seqlens`` is None).
+    Empty sequences contribute nothing; rows outside every sequence are not allowed
+    (``cu_seqlens`` must run from 0 to T)."""
     x, ref = _f64(x), _f64(ref)
+    if x.shape != ref.shape or ref.ndim != 3:
+        raise ValueError(f"x and ref must share one [T, H, D] shape: {x.shape} vs {ref.shape}")
     T, H, _ = ref.shape
     cu = _cu(cu_seqlens, T)
+    if cu.ndim != 1 or len(cu) < 2 or cu[0] != 0 or cu[-1] != T or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must be non-decreasing from 0 to T")
     worst = 0.0
     for s in range(len(cu) - 1):
         a, b = int(cu[s]), int(cu[s + 1])
         if b == a:
             continue
         for h in range(H):
-            worst = max(worst, rel_l2(x[a:b, h], ref[a:b, h]))
+            worst = _worse(worst, rel_l2(x[a:b, h, :], ref[a:b, h, :]))
+    return worst
+
+
+def max_rel_l2_per_state(x, ref) -> float:
+    """Maximum over (sequence, head) of the relative L2 error on ``[S, H, D, D]``
+    states.  A zero reference state (an empty sequence) must be matched exactly:
+    any non-zero value there gives inf."""
+    x, ref = _f64(x), _f64(ref)
+    if x.shape != ref.shape or ref.ndim != 4:
+        raise ValueError(f"x and ref must share one [S, H, D, D] shape: {x.shape} vs {ref.shape}")
+    S, H = ref.shape[:2]
+    worst = 0.0
+    for s in range(S):
+        for h in range(H):
+            worst = _worse(worst, rel_l2(x[s, h], ref[s, h]))
     return worst

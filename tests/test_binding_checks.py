@@ -91,3 +91,53 @@ def test_chunk_state_and_prefix_shapes():
         api.state_prefix(g, 1, out=f32(2, 2, 64, 32))
     with pytest.raises(ValueError, match="gathered must be"):
         api.state_prefix(f32(2, 2, 64, 64), 1)
+
+
+def test_one_device_per_call():
+    """Every tensor of a call must be on q's device (the library launches there); a
+    tensor elsewhere is rejected before the library is reached.  ``meta`` tensors stand
+    in for a second device."""
+    q = bf(10, 2, 64)
+    other = torch.zeros((10, 2, 64), dtype=torch.bfloat16, device="meta")
+    with pytest.raises(ValueError, match="is on meta"):
+        api.prefill(q, other, q, beta=64)
+    with pytest.raises(ValueError, match="is on meta"):
+        api.prefill(q, q, q, beta=64, out=other)
+    with pytest.raises(ValueError, match="is on meta"):
+        api.prefill(q, q, q, beta=64, state_out=torch.zeros((1, 2, 64, 64), device="meta"))
+    with pytest.raises(ValueError, match="is on meta"):
+        api.prefill(q, q, q, beta=64, initial_state=torch.zeros((1, 2, 64, 64), device="meta"))
+    qd = bf(3, 2, 64)
+    with pytest.raises(ValueError, match="is on meta"):
+        api.decode_step(qd, qd, qd, torch.zeros((3, 2, 64, 64), device="meta"))
+    ws = f32(4, 2, 64, 64)
+    with pytest.raises(ValueError, match="is on meta"):
+        api.state_out(ws, torch.zeros((4, 2, 64, 64), device="meta"))
+    with pytest.raises(ValueError, match="is on meta"):
+        api.state_out(ws, f32(4, 2, 64, 64), torch.zeros(4, dtype=torch.int32, device="meta"))
+    with pytest.raises(ValueError, match="is on meta"):
+        api.chunk_state(q, other)
+    with pytest.raises(ValueError, match="is on meta"):
+        api.state_prefix(f32(2, 1, 2, 64, 64), 1, out=torch.zeros((1, 2, 64, 64), device="meta"))
+
+
+def test_overlapping_state_buffers():
+    """initial_state is copied into a separate state_out before the in-place update, so
+    two views that overlap without coinciding would corrupt it: rejected."""
+    q = bf(10, 2, 64)
+    n = 2 * 64 * 64
+    buf = f32(3 * n)
+    init = buf[:2 * n].view(2, 2, 64, 64)
+    shifted = buf[n:3 * n].view(2, 2, 64, 64)
+    with pytest.raises(ValueError, match="overlap"):
+        api.prefill(q, q, q, beta=64, cu_seqlens=[0, 4, 10], initial_state=init, state_out=shifted)
+    with pytest.raises(Reached):       # the same tensor: an in-place update, allowed
+        api.prefill(q, q, q, beta=64, cu_seqlens=[0, 4, 10], initial_state=init, state_out=init)
+    with pytest.raises(Reached):       # disjoint
+        api.prefill(q, q, q, beta=64, cu_seqlens=[0, 4, 10], initial_state=init,
+                    state_out=f32(2, 2, 64, 64))
+    with pytest.raises(ValueError, match="overlap"):
+        api.state_out(init, shifted)
+    g = f32(3, 1, 2, 64, 64)
+    with pytest.raises(ValueError, match="overlap"):
+        api.state_prefix(g, 1, out=g[1])

@@ -22,15 +22,7 @@ IDS = [f"{'bf16' if d == torch.bfloat16 else 'fp32'}-d{D}" for d, D in CASES]
 
 
 def _state_err(st_gpu, st_ref):
-    worst = 0.0
-    S, H = st_ref.shape[:2]
-    for s in range(S):
-        for h in range(H):
-            if np.any(st_ref[s, h]):
-                worst = max(worst, oracle.rel_l2(st_gpu[s, h], st_ref[s, h]))
-            else:
-                assert float(np.abs(st_gpu[s, h]).max()) == 0.0
-    return worst
+    return oracle.max_rel_l2_per_state(st_gpu, st_ref)
 
 
 @pytest.mark.parametrize("dtype,D", CASES, ids=IDS)

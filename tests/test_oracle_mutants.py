@@ -36,6 +36,8 @@ def test_mutant_is_caught(mid, tmp_path):
         for pin in oracle_pins.ALL_PINS:
             try:
                 pin()
-            except AssertionError:
+            except (AssertionError, ValueError):
+                # ValueError: the broken build produced a non-finite value, which the
+                # error metric refuses to compare (every pin passes on the real build)
                 failed.append(pin.__name__)
     assert failed, f"no pin catches mutant {mid}: {MUTANTS[mid]}"

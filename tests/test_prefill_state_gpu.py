@@ -31,12 +31,7 @@ IDS = [f"{'bf16' if d == torch.bfloat16 else 'fp32'}-b{b}-d{D}" for d, b, D in K
 
 
 def _state_err(st_gpu, st_ref):
-    worst = 0.0
-    S, H = st_ref.shape[:2]
-    for s in range(S):
-        for h in range(H):
-            worst = max(worst, oracle.rel_l2(st_gpu[s, h], st_ref[s, h]))
-    return worst
+    return oracle.max_rel_l2_per_state(st_gpu, st_ref)
 
 
 @pytest.mark.parametrize("dtype,beta,D", KERNELS, ids=IDS)
