@@ -33,6 +33,8 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -392,6 +394,11 @@ def run_ours(args):
         line["e2e"] = e2e_prefill(args, api, torch, q, k, v, B, N, H, D, beta, world, dev)
         line["decode"], dctx = bench_decode(api, synth, torch, dev, stream, peak_bw, rank, world)
         line["concurrent"] = bench_concurrent(api, torch, stream, dctx, q, k, v, o, beta, world)
+        if rank == 0 and world == 1:  # the host baseline is a 1-GPU figure
+            try:
+                line["decode"]["cpu_baseline"] = decode_cpu_baseline(torch, dctx)
+            except Exception as e:  # an extra that fails must not cost the main line
+                line["decode"]["cpu_baseline"] = {"error": repr(e)}
         del dctx
         line["lasp_chunk_state"] = bench_chunk_state(api, torch, stream, k, v, peak_bw, world)
         if world == 1:  # rank-local extra: no collective, so a failure cannot strand other ranks
@@ -403,6 +410,15 @@ def run_ours(args):
                 line["prefill_options"] = bench_prefill_options(api, torch, stream, q, k, v, o, peak_bw)
             except Exception as e:
                 line["prefill_options"] = {"error": repr(e)}
+            try:
+                line["headline_repeat"] = bench_headline_repeat(api, torch, stream, q, k, v, o, beta,
+                                                                peak_bw, torch.cuda.current_device())
+            except Exception as e:
+                line["headline_repeat"] = {"error": repr(e)}
+            try:
+                line["configs"] = bench_configs(api, synth, torch, stream, dev, peaks, cpu=(rank == 0))
+            except Exception as e:
+                line["configs"] = {"error": repr(e)}
     if rank == 0 and world == 1 and not args.no_extras:  # the host baseline is a 1-GPU figure
         line["cpu_baseline"] = cpu_baseline(B, N, H, D, beta)
     if world > 1:
@@ -567,6 +583,189 @@ def bench_prefill_options(api, torch, stream, q, k, v, o, peak_bw, reps=10, warm
                      "status": api.status_string(api.device_status(stream))}
     res["launches_per_option"] = reps
     return res
+
+
+def timed_launches(torch, stream, fn, reps, warm, device_index):
+    """Per-launch CUDA-event times (ms) of ``fn`` on ``stream`` after ``warm`` untimed calls,
+    with the SM clock sampled while they run."""
+    for _ in range(warm):
+        fn()
+    stream.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    with ClockSampler(device_index, period_s=0.005) as clk:
+        ev[0].record(stream)
+        for i in range(reps):
+            fn()
+            ev[i + 1].record(stream)
+        stream.synchronize()
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)], clk.summary()
+
+
+def spread(ms):
+    """Median and range of per-launch times."""
+    return {"median": statistics.median(ms), "min": min(ms), "max": max(ms), "launches": len(ms)}
+
+
+def tiled_flops_packed(lengths, H: int, D: int, beta: int) -> int:
+    """Tiled-form flops of a packed batch: every block of beta tokens counted in full
+    (a partial last block costs a whole block): per block 4 beta^2 D + 4 beta D^2 per head."""
+    blocks = sum((n + beta - 1) // beta for n in lengths)
+    return blocks * H * (4 * beta * beta * D + 4 * beta * D * D)
+
+
+def prefill_leg(name, ms, clocks, T, H, D, flops, peaks):
+    """Metric view of one timed prefill configuration."""
+    s = statistics.median(ms) / 1e3
+    bw = prefill_bytes(T, H, D) / s / 1e9
+    tf = flops / s / 1e12
+    return {"workload": name, "ms_per_launch": spread(ms), "tokens_per_s": T / s,
+            "tflops_tiled": tf, "pct_bf16_peak": 100.0 * tf / float(peaks["bf16_tflops"]),
+            "hbm_gbs": bw, "hbm_frac": bw / float(peaks["hbm_gbs"]),
+            "algorithmic_bytes": prefill_bytes(T, H, D), "clocks": clocks}
+
+
+def cpu_oracle_quadratic(q, k, v, reps=20):
+    """The fp64 quadratic-form oracle on a whole (tiny) workload, mean of ``reps`` runs."""
+    import oracle
+    cores = max(1, os.cpu_count() or 1)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.quadratic(q, k, v, nthreads=cores)
+    t = (time.perf_counter() - t0) / reps
+    T, H = q.shape[0], q.shape[1]
+    return {"value": T / t, "unit": "tokens/s", "cores": min(cores, H), "kind": "oracle", "seconds": t,
+            "sample": f"fp64 quadratic form, the whole workload ({H} heads x {T} tokens), mean of {reps} runs"}
+
+
+def cpu_oracle_prefill(q, k, v, cu, rmsnorm, heads, what):
+    """The fp64 recurrent oracle on the first ``heads`` heads of a workload, all its tokens,
+    on the host cores; value in tokens/s of the H-head layer."""
+    import oracle
+    H = q.shape[1]
+    cores = max(1, os.cpu_count() or 1)
+    t0 = time.perf_counter()
+    oracle.recurrent(q[:, :heads], k[:, :heads], v[:, :heads], cu, rmsnorm=rmsnorm,
+                     want_o=True, nthreads=cores)
+    t = time.perf_counter() - t0
+    T = q.shape[0]
+    S = 1 if cu is None else len(cu) - 1
+    return {"value": T * heads / H / t, "unit": "tokens/s", "cores": min(cores, heads * S),
+            "kind": "oracle", "seconds": t,
+            "sample": f"fp64 recurrent form, {what}: {heads}/{H} heads x all {T} tokens, "
+                      f"value = token-heads / {H} / time"}
+
+
+def bench_configs(api, synth, torch, stream, dev, peaks, cpu: bool):
+    """The other configurations of the method's workload list, each timed on its own:
+    the tiny fp32 case, the MiniMax-layer prefill (64 heads x 128, N = 8192, RMSNorm,
+    beta = 128 and 64), the packed varlen batch (262144 tokens, 8 seeded sequences) and a
+    mixed batch of one-token (decode) rows and prefill chunks from per-sequence states."""
+    di = dev.index if dev.index is not None else torch.cuda.current_device()
+    res = {}
+    # config 1: B=1, H=2, N=256, D=64, beta=64, fp32, no norm
+    q, k, v = synth.qkv(256, 2, 64, seed=0, dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    ms, clk = timed_launches(torch, stream, lambda: api.prefill(q, k, v, beta=64, out=o, stream=stream),
+                             200, 5, di)
+    res["c1_tiny_fp32"] = {"workload": "B=1, H=2, N=256, D=64, beta=64, fp32, no norm",
+                           "ms_per_launch": spread(ms), "tokens_per_s": 256 / (statistics.median(ms) / 1e3),
+                           "clocks": clk}
+    if cpu:
+        res["c1_tiny_fp32"]["cpu_baseline"] = cpu_oracle_quadratic(q, k, v)
+    # config 2: MiniMax layer, RMSNorm, beta 128 and 64
+    N, H, D = 8192, 64, 128
+    q, k, v = synth.qkv(N, H, D, seed=2, dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q)
+    c2 = {}
+    for beta in (128, 64):
+        ms, clk = timed_launches(torch, stream, lambda: api.prefill(q, k, v, beta=beta, rmsnorm=True, out=o,
+                                                                    stream=stream), 50, 5, di)
+        c2[f"beta{beta}"] = prefill_leg(f"B=1, N={N}, H={H}, D={D}, beta={beta}, bf16, RMSNorm", ms, clk,
+                                        N, H, D, tiled_flops_packed([N], H, D, beta), peaks)
+    if cpu:
+        c2["cpu_baseline"] = cpu_oracle_prefill(q, k, v, None, True, H, "config 2 with RMSNorm")
+    res["c2_layer_rmsnorm"] = c2
+    del q, k, v, o
+    # config 4: packed varlen, 262144 tokens, 8 seeded sequences, beta = 128
+    T, S = 262144, 8
+    cu = synth.cu_seqlens_uniform(T, S, seed=0)
+    lens = [int(cu[i + 1] - cu[i]) for i in range(S)]
+    q, k, v = synth.qkv(T, H, D, seed=4, dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q)
+    ms, clk = timed_launches(torch, stream, lambda: api.prefill(q, k, v, beta=128, cu_seqlens=cu, out=o,
+                                                                stream=stream), 20, 3, di)
+    c4 = prefill_leg(f"packed varlen, T={T}, S={S} seeded uniform lengths {lens}, H={H}, D={D}, "
+                     f"beta=128, bf16", ms, clk, T, H, D, tiled_flops_packed(lens, H, D, 128), peaks)
+    if cpu:
+        c4["cpu_baseline"] = cpu_oracle_prefill(q, k, v, cu, False, min(H, 4), "config 4")
+    res["c4_packed_varlen"] = c4
+    del q, k, v, o
+    # mixed batch: 256 one-token rows and 8 chunks of 4096 tokens, each from its own state,
+    # in one la_prefill; against the one-token rows through la_decode_step plus the chunks
+    # through la_prefill
+    n1, nc, L = 256, 8, 4096
+    lens = [1] * n1 + [L] * nc
+    cu_m = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Tm = int(cu_m[-1])
+    q, k, v = synth.qkv(Tm, H, D, seed=6, dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q)
+    X = synth.initial_state(n1 + nc, H, D, tokens=4096, seed=6, device=dev)
+    st = X.clone()
+    ms_mix, clk = timed_launches(torch, stream, lambda: api.prefill(
+        q, k, v, beta=128, cu_seqlens=cu_m, initial_state=st, state_out=st, out=o, stream=stream), 20, 3, di)
+    qd, kd, vd = (x[:n1].contiguous() for x in (q, k, v))
+    od = torch.empty_like(qd)
+    st1 = X[:n1].clone()
+    qc, kc, vc = (x[n1:].contiguous() for x in (q, k, v))
+    oc = torch.empty_like(qc)
+    stc = X[n1:].clone()
+    cu_c = [0] + [L * (i + 1) for i in range(nc)]
+
+    def split():
+        api.decode_step(qd, kd, vd, st1, out=od, stream=stream)
+        api.prefill(qc, kc, vc, beta=128, cu_seqlens=cu_c, initial_state=stc, state_out=stc, out=oc,
+                    stream=stream)
+    ms_split, _ = timed_launches(torch, stream, split, 20, 3, di)
+    res["f4_mixed_batch"] = {
+        "workload": f"{n1} one-token sequences + {nc} chunks of {L} tokens, H={H}, D={D}, bf16, "
+                    f"each from its own state (read and written in place)",
+        "one_prefill_launch_ms": spread(ms_mix),
+        "decode_step_plus_prefill_ms": spread(ms_split),
+        "clocks": clk,
+        "note": "the same work as one la_prefill launch, and as la_decode_step for the one-token "
+                "rows followed by la_prefill for the chunks (two launches)"}
+    res["status"] = api.status_string(api.device_status(stream))
+    return res
+
+
+def bench_headline_repeat(api, torch, stream, q, k, v, o, beta, peak_bw, device_index, reps=100):
+    """The main step repeated: the spread of the per-launch time over ``reps`` launches and
+    the SM clock while they ran."""
+    ms, clk = timed_launches(torch, stream, lambda: api.prefill(q, k, v, beta=beta, out=o, stream=stream),
+                             reps, 3, device_index)
+    H, D = q.shape[-2], q.shape[-1]
+    T = q.numel() // (H * D)
+    med = statistics.median(ms)
+    return {"ms_per_launch": spread(ms), "hbm_frac_median": prefill_bytes(T, H, D) / (med / 1e3) / 1e9 / peak_bw,
+            "clocks": clk, "status": api.status_string(api.device_status(stream))}
+
+
+def decode_cpu_baseline(torch, dctx, Bs=16):
+    """The fp64 decode oracle over the 64 decode steps on the first ``Bs`` sequences of the
+    decode batch (all heads), from the GPU state before the steps; tokens/s of the batch."""
+    import oracle
+    dstream, state0, toks, _ = dctx
+    st = state0[:Bs].detach().to("cpu").double().numpy()
+    cores = max(1, os.cpu_count() or 1)
+    t0 = time.perf_counter()
+    for t in range(len(toks)):
+        q, k, v = (x[:Bs] for x in toks[t])
+        _, st = oracle.decode_step(q, k, v, st, nthreads=cores)
+    sec = time.perf_counter() - t0
+    B = state0.shape[0]
+    return {"value": Bs * len(toks) / sec, "unit": "decode tokens/s", "cores": cores, "kind": "oracle",
+            "seconds": sec, "sample": f"fp64 decode oracle, {len(toks)} steps on {Bs}/{B} sequences x all "
+                                      f"heads, from a copy of the GPU decode state"}
 
 
 def bench_chunk_state(api, torch, stream, k, v, peak_bw, world, reps=5):

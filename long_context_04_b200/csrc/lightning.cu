@@ -124,12 +124,6 @@ la_status launch_tc(const PrefillTcParams &p, int units, cudaStream_t stream) {
 
 la_status launch_pair(const la::PrefillPairParams &p, int pairs, cudaStream_t stream) {
     using C = la::PairCfg;
-    // Ring depths.  CTA 0's group P waits on full_kv of a partial last block b; its parity
-    // wait is exact only if the slot's previous load (block b - NKV) is known to have landed
-    // when the wait starts.  Group P knows it through S_b (issued after issuer A waited on
-    // the loads of blocks up to b - SAHEAD) or through P_{b-NPB} V (issuer B waited on the
-    // loads up to b - NPB), so one of the two must reach back far enough.
-    static_assert(C::SAHEAD <= C::NKV || C::NPB <= C::NKV, "ring depths: group P's tail wait");
     auto kern = la::prefill_pair_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
@@ -227,7 +221,8 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
             la::PrefillPairParams pp;
             std::memset(&pp, 0, sizeof pp);
             if (!make_map(&pp.tmap_q64, q, Tm, H, D, 64) || !make_map(&pp.tmap_k64, k, Tm, H, D, 64) ||
-                !make_map(&pp.tmap_k128, k, Tm, H, D, 128) || !make_map(&pp.tmap_v128, v, Tm, H, D, 128))
+                !make_map(&pp.tmap_k128, k, Tm, H, D, 128) || !make_map(&pp.tmap_v128, v, Tm, H, D, 128) ||
+                !make_map(&pp.tmap_o32, o, Tm, H, D, 32))
                 return LA_ERR_CUDA;
             pp.o = static_cast<__nv_bfloat16 *>(o);
             pp.state = state;

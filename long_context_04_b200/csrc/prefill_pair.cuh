@@ -1,45 +1,48 @@
 // Lightning-attention prefill, beta = 128 and D = 128, bf16: one CTA pair per
 // (sequence, head), paired tcgen05 MMAs (cta_group::2).
 //
-// Same block algorithm as prefill_tc.cuh (MiniMax-01, "Scaling Foundation
-// Models with Lightning Attention"; CSDN digest section 2.1, mizuki blog
-// appendix "key concepts"): per block b of 128 tokens,
-//     O_b = [(Q_b K_b^T) (.) M] V_b + Q_b KV,     KV += K_b^T V_b.
+// Block algorithm (MiniMax-01, "Scaling Foundation Models with Lightning
+// Attention"; CSDN digest section 2.1, mizuki blog appendix "key concepts"): per
+// block b of 128 tokens of one sequence and head,
+//     O_b = [(Q_b K_b^T) (.) M] V_b + Q_b KV,     KV += K_b^T V_b,
+// with the causal 0/1 mask M (j <= i), KV reset at the sequence start (or set to
+// an initial state), and an optional RMSNorm of each output row.
 //
-// Work split inside the pair (CTA rank c = 0 or 1): every MMA is an M = 128,
-// N = 128 paired MMA issued by one thread of CTA 0.  Each CTA supplies half of
-// the A rows and half of the B rows from its own shared memory and receives
-// its half of the D rows, for all N columns, in its own TMEM:
-//   S   = Q K^T      A: own 64 query rows    B: own 64 key rows      D: own rows x 128 keys
-//   O   = P V        A: own 64 rows of P     B: own 64 value columns D: own rows x 128 columns
-//   O  += Q snap     A: own 64 query rows    B: own 64 rows of KV^T  D: (the same O)
-//   dKV^T = V^T K    A: own 64 value columns B: own 64 key dims      D: own 64 value cols x 128 dims
-// so a CTA stages only its halves (64 KB per block instead of 80 KB for the
-// unpaired kernel) and each tensor-core operand byte is read once per pair
-// instead of once per CTA.  The halves arrive through three TMA rings (key
-// rows 2 deep, query rows 4 deep, key dims + value columns 2 deep), each slot
-// released by the last MMA that reads it.  Each CTA keeps
-// its 64 columns of the fp32 state, transposed (KV^T[j][i]), in epilogue
-// registers, and its output rows are complete (all 128 columns) inside the
-// CTA, so the RMSNorm needs no exchange between the CTAs.
+// Products per block (CTA rank c = 0 or 1).  Every MMA is paired: M = 128 with
+// 64 rows per CTA; each CTA supplies half of the B rows from its own shared
+// memory and receives its 64 D rows, for all N columns, in its own TMEM:
+//   F1 = [S_b | O_b] = Q_b [K_b ; snap_b]^T   N = 256, K = dims
+//          A: own 64 query rows     B: own 64 key rows, then own 64 rows of KV^T
+//   O_b += P_b V_b                           N = 128, K = keys
+//          A: own 64 rows of P      B: own 64 value columns
+//   dKV_b^T = V_b^T K_b                      N = 128, K = tokens
+//          A: own 64 value columns  B: own 64 key dims
+// F1 gives the intra-block scores and the inter-block term Q_b KV_{<b} in one
+// product: both have Q_b as their A operand, so K_b and the bf16 snapshot of the
+// state stack into one 128-row B tile.  An N = 256 paired MMA keeps the tensor
+// pipe busy for about as long as one thread takes to issue a tcgen05.mma.  The
+// accumulators use the folded layout of an M = 64-per-CTA MMA: lanes 0..63 hold
+// the CTA's 64 rows for the N columns the even CTA supplies, lanes 64..127 the
+// same rows for the odd CTA's columns.  So F1 leaves S in the first 64 TMEM
+// columns of its region and O in the next 64, exactly where the N = 128 product
+// P V accumulates.
 //
-// The paired accumulators use the folded TMEM layout of an M = 64-per-CTA
-// MMA: lanes 0..63 hold the 64 rows for columns [0, N/2), lanes 64..127 the
-// same rows for columns [N/2, N), both in TMEM columns [0, N/2).
+// Schedule.  Two issuing threads: one issues dKV_0, dKV_1, ... as soon as each
+// block's key dims and values have landed (the state chain runs ahead of F1), the
+// other issues F1_0, then per block b: F1_{b+1}, P_b V_b.  The snapshot F1_{b+1}
+// needs (from dKV_b) and the P_b that P_b V_b needs (from F1_b) are produced by
+// the epilogue while the other products run.
 //
-// Warps (352 threads per CTA):
-//   warp 0      TMA producer: each CTA loads its own halves; CTA 1's loads complete
-//               CTA 0's ring barriers directly (the .cta_group::2 load form)
-//   warp 1      CTA 0: TMEM owner and MMA issuer A: S_{b+1} (look-ahead), dKV_b^T = V_b^T K_b.
-//               CTA 1: takes part in the TMEM allocation only.
-//   warps 2..5  group P: S -> causal mask -> bf16 P (shared memory, A operand of P V)
-//   warps 6..9  group O: KV^T += dKV^T, bf16 snapshot, O -> (RMSNorm) -> bf16 store,
-//               final fp32 state -> global store
-//   warp 10     CTA 0: MMA issuer B: O_b = Q_b snap(KV_{<b}), O_b += P_b V_b.
-// Two issuing threads keep the tensor pipe fed; each has one commit per block
-// (s_full and kv_done for A, o_done for B), and each commit arrives on the
-// barriers of both CTAs.  Signals to the issuers are mbarrier arrivals (remote
-// ones from CTA 1).  Every wait is bounded; on a timeout the CTA records
+// Warps (480 threads per CTA):
+//   warp 0       TMA producer (both CTAs)
+//   warp 1       TMEM owner (both CTAs); CTA 0: issuer of F1 and P V
+//   warps 2..5   group P (S -> causal mask -> bf16 P in shared memory)
+//   warps 6..9   group KV (KV^T += dKV^T in registers, bf16 snapshot into the key-row
+//                slot of the next block, final state)
+//   warps 10..13 group O (O -> optional RMSNorm -> bf16, TMA store)
+//   warp 14      CTA 0: issuer of dKV
+// Each epilogue group has one warp per TMEM sub-partition (warp w reads lanes
+// 32 (w mod 4) .. + 31).  Every wait is bounded; on a timeout the CTA records
 // DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
 
@@ -52,6 +55,7 @@ struct PrefillPairParams {
     CUtensorMap tmap_k64;   // K, box 64 x 64
     CUtensorMap tmap_k128;  // K, box 64 x 128
     CUtensorMap tmap_v128;  // V, box 64 x 128
+    CUtensorMap tmap_o32;   // O, box 64 x 32 (stores)
     __nv_bfloat16 *o;
     float *state;           // [S][H][D][D] or nullptr: final states
     const float *state_in;  // [S][H][D][D] or nullptr: initial states (may alias state)
@@ -61,96 +65,72 @@ struct PrefillPairParams {
     SeqTable seqs;
 };
 
-#ifndef LA_PAIR_S_AHEAD
-#define LA_PAIR_S_AHEAD 1
-#endif
-#ifndef LA_PAIR_P_BUFS
-#define LA_PAIR_P_BUFS 1
-#endif
-#ifndef LA_PAIR_KK_DEPTH
-#define LA_PAIR_KK_DEPTH 2
-#endif
-#ifndef LA_PAIR_QH_DEPTH
-#define LA_PAIR_QH_DEPTH 4
-#endif
-#ifndef LA_PAIR_KV_DEPTH
-#define LA_PAIR_KV_DEPTH 2
-#endif
-
 struct PairCfg {
     static constexpr int BETA = 128, D = 128;
     static constexpr int HBOX = 64 * 128;               // 64 rows x 128 B
     static constexpr int FBOX = 128 * 128;              // 128 rows x 128 B
-    // Three TMA rings, each released at the last use of its tiles (all tiles
-    // 128-byte swizzled; a "half" is dims [0,64) | [64,128) of 64 rows):
-    //   KK: own 64 key rows, both dim halves           (S = Q K^T)
-    //   QH: own 64 query rows, both dim halves         (S, and O += Q snap)
-    //   KV: 128 key rows x own 64 dims | 128 value rows x own 64 columns (P V, V^T K)
-    static constexpr int NKK = LA_PAIR_KK_DEPTH, NQH = LA_PAIR_QH_DEPTH, NKV = LA_PAIR_KV_DEPTH;
-    // ring of block-completion barriers; a ring's depth may not exceed the barrier
-    // ring it waits on, or a phase could be lapped before its waiter sees it
-    static constexpr int NDONE = 4;
-    // S runs SAHEAD blocks ahead of the block whose P V consumes it, in a ring of
-    // SAHEAD + 1 TMEM buffers (the extra one is being turned into P by group P)
-    static constexpr int SAHEAD = LA_PAIR_S_AHEAD, NS = SAHEAD + 1;
-    static_assert(NKK <= NS, "key-row slots are released by s_full[NS]");
-    static_assert(NQH <= NDONE && NKV <= NDONE, "slot release ring");
-    static constexpr int KK_BYTES = 2 * HBOX, QH_BYTES = 2 * HBOX, KV_BYTES = 2 * FBOX;
-    static constexpr int OFF_KK = 0;
-    static constexpr int OFF_QH = OFF_KK + NKK * KK_BYTES;
-    static constexpr int OFF_KV = OFF_QH + NQH * QH_BYTES;
-    static constexpr int KV_OFF_VC = FBOX;               // within a KV stage
-    // P buffers (own 64 rows of P, keys [0,64) | [64,128)); P_b goes to buffer b % NPB
-    static constexpr int NPB = LA_PAIR_P_BUFS, P_BYTES = 2 * HBOX;
-    static_assert(NPB <= NDONE, "P buffers are released by o_done");
-    static constexpr int OFF_P = OFF_KV + NKV * KV_BYTES;
-    // two bf16 snapshots of the state (own 64 rows of KV^T, dims [0,64) | [64,128)):
-    // the one for block b+1 is written while O_b = Q_b snap still reads the other
-    static constexpr int SNAP_BYTES = 2 * HBOX;
-    static constexpr int OFF_SNAP = OFF_P + NPB * P_BYTES;
-    static constexpr int OFF_MISC = OFF_SNAP + 2 * SNAP_BYTES;
+    // Shared-memory rings (128-byte swizzled tiles; a "half" is dims or columns
+    // [0,64) | [64,128)), each slot released by the product that reads it last:
+    //   Q : own 64 query rows, both dim halves (A of F1)                     f1_done
+    //   KS: per dim half 128 rows: own 64 key rows (TMA), then own 64 rows of
+    //       the snapshot KV^T (group KV) (B of F1)                           f1_done
+    //   KD: 128 key rows x own 64 dims (B of dKV^T)                          dkv_done
+    //   V : 128 value rows x own 64 columns (A of dKV^T, B of P V)           o_done
+    //   P : own 64 rows of P, both key halves (A of P V)                     o_done
+    // (a value tile is released by P V, which follows its dKV in every schedule)
+    static constexpr int NQ = 2, NKS = 2, NKD = 2, NV = 3, NPB = 2;
+    static constexpr int NF = 3;                        // F1 TMEM regions (S | O)
+    static constexpr int NDK = 2;                       // dKV TMEM buffers
+    // A ring's slot of block x is tested free on the done barrier of block x, which
+    // must not have been lapped (by block x + ring size) when the producer tests it.
+    static_assert(NQ <= NF && NKS <= NF && NV <= NF && NKD <= NDK && NPB <= NF, "release rings");
+    static constexpr int Q_BYTES = 2 * HBOX, KS_BYTES = 2 * FBOX, T_BYTES = FBOX;
+    static constexpr int P_BYTES = 2 * HBOX;
+    static constexpr int OST_BYTES = 32 * 128;          // one 32-row x 64-column O box
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KS = OFF_Q + NQ * Q_BYTES;
+    static constexpr int OFF_KD = OFF_KS + NKS * KS_BYTES;
+    static constexpr int OFF_V = OFF_KD + NKD * T_BYTES;
+    static constexpr int OFF_P = OFF_V + NV * T_BYTES;
+    static constexpr int OFF_OST = OFF_P + NPB * P_BYTES;
+    static constexpr int OFF_MISC = OFF_OST + 4 * OST_BYTES;
     static constexpr int MISC = 2048;
     static constexpr int SMEM_BYTES = 1024 + OFF_MISC + MISC;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-    // TMEM columns: S[NS], O[2], dKV[2], 64 columns each (folded layout)
-    static constexpr int TM_S = 0, TM_O = 64 * NS, TM_DKV = 64 * NS + 128;
-    static_assert(TM_DKV + 128 <= 512, "TMEM columns");
+    // TMEM columns: F1 region f = [S (64) | O (64)] at 128 f, then the dKV buffers
+    static constexpr int TM_F1 = 0, TM_DKV = 128 * NF;
+    static_assert(TM_DKV + 64 * NDK <= 512, "TMEM columns");
     static constexpr int TMEM_COLS = 512;
     static constexpr int GROUP = 128;
-    static constexpr int WARP_B = 10;                   // second MMA issuer (CTA 0)
-    static constexpr int THREADS = 64 + 2 * GROUP + 32;
-    static constexpr uint32_t ID_S = idesc_bf16_f32(128, 128, 0, 0);
+    static constexpr int WARP_D = 14;                   // issuer of dKV (CTA 0)
+    static constexpr int THREADS = 64 + 3 * GROUP + 32;
+    static constexpr uint32_t ID_F1 = idesc_bf16_f32(128, 256, 0, 0);
     static constexpr uint32_t ID_PV = idesc_bf16_f32(128, 128, 0, 1);
-    static constexpr uint32_t ID_QKV = idesc_bf16_f32(128, 128, 0, 0);
     static constexpr uint32_t ID_KV = idesc_bf16_f32(128, 128, 1, 1);
 };
 
-// Every wait below is a parity wait on one phase x of a barrier.  Two rules make
-// it exact: phase x - 1 is known to be complete when the wait starts (the waiter
-// saw it, or a chain of signals implies it), and phase x + 1 cannot complete
-// before the wait returns.  This is why the S buffers, the P buffers and the
-// snapshots have a barrier per buffer and the tail zeroing a single-phase barrier.
+// Every wait below is a parity wait on one phase x of a barrier.  Two rules make it
+// exact: phase x - 1 is known complete when the wait starts, and phase x + 1 cannot
+// complete before the wait returns (argued for each barrier where it is waited on).
 struct PairMisc {
-    // Ring barriers.  "full" barriers are used in CTA 0 only: CTA 0's producer
-    // expects the bytes of both CTAs and CTA 1's loads complete them directly.
-    // A slot is free again once the MMAs reading it have completed: s_full[j % NS]
-    // frees key-row slot j (S_j done), o_done[j % 4] the query slot (O_j done, which
-    // follows S_j), o_done and kv_done[j % 4] together the K/V slot.  Every MMA
-    // commit arrives on the barrier of both CTAs.
-    uint64_t full_kk[PairCfg::NKK];
-    uint64_t full_qh[PairCfg::NQH];
-    uint64_t full_kv[PairCfg::NKV];
-    uint64_t tail_kv;              // CTA 1: its own KV tiles of a partial last block landed
+    // used in CTA 0: TMA completion (CTA 1's loads complete them directly)
+    uint64_t full_q[PairCfg::NQ];
+    uint64_t full_ks[PairCfg::NKS];
+    uint64_t full_kd[PairCfg::NKD];
+    uint64_t full_v[PairCfg::NV];
+    uint64_t tail_v;               // CTA 1: its own value tile of a partial last block landed
     uint64_t tail_zeroed;          // used in CTA 0: value rows past the sequence end zeroed
-    uint64_t s_full[PairCfg::NS];  // S_j complete (buffer j % NS)
-    uint64_t s_free[PairCfg::NS];  // used in CTA 0: group P of both CTAs has loaded S_j
-    uint64_t kv_done[4];           // dKV_j complete (issuer A)
-    uint64_t o_done[4];            // O_j complete (issuer B)
-    uint64_t o_free[2];            // used in CTA 0: arrivals from both CTAs
-    uint64_t dkv_free[2];
-    uint64_t p_ready[PairCfg::NPB];  // used in CTA 0: P_j stored in buffer j % NPB
-    uint64_t snap_ready[2];        // used in CTA 0: snapshot u (for block u) in buffer u % 2
+    // MMA completion (each commit arrives in both CTAs)
+    uint64_t f1_done[PairCfg::NF];   // F1_j complete (region j % NF)
+    uint64_t dkv_done[PairCfg::NDK]; // dKV_j complete (buffer j % NDK)
+    uint64_t o_done[PairCfg::NF];    // P_j V_j complete (region j % NF)
+    // used in CTA 0: epilogue -> issuers (arrivals from both CTAs)
+    uint64_t f1_free[PairCfg::NF];   // groups P and O have loaded S_j and O_j
+    uint64_t dkv_free[PairCfg::NDK]; // group KV has loaded dKV_j
+    uint64_t p_ready[PairCfg::NPB];  // P_j stored in buffer j % NPB
+    uint64_t snap_ready[PairCfg::NKS];  // snapshot u (the state before block u) in slot u % NKS
     uint64_t drain;
+    uint64_t done0;                // phase 0 completed at the start: a wait that always passes
     uint64_t ss_bar[2];            // group O: RMSNorm partial sums written (per block parity)
     uint32_t tmem_base;
     int abort_flag;
@@ -175,36 +155,35 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     int seq_start, seq_len, sid;
     p.seqs.get(rank, seq_start, seq_len, sid);
     const int nb = (seq_len + C::BETA - 1) / C::BETA;
-    // a partial last block: its value rows past the sequence end are zeroed by group P
+    // a partial last block: its value rows past the sequence end are zeroed by group KV
     const bool tail = nb > 0 && seq_len < nb * C::BETA;
-    // Snapshot u of the state (bf16, buffer u % 2) feeds O_u = Q_u snap_u.  With an
-    // initial state X the first one (u = 0) is X; without one, block 0 has no
-    // inter-block term and the first snapshot is u = 1.
-    const int u0 = p.state_in != nullptr ? 0 : 1;
     const uint64_t tlimit = p.timeout_ns;
     volatile int *abort_flag = &m->abort_flag;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::NKK; ++s) mbar_init(&m->full_kk[s], 1);
-        for (int s = 0; s < C::NQH; ++s) mbar_init(&m->full_qh[s], 1);
-        for (int s = 0; s < C::NKV; ++s) mbar_init(&m->full_kv[s], 1);
-        for (int s = 0; s < C::NS; ++s) {
-            mbar_init(&m->s_full[s], 1);
-            mbar_init(&m->s_free[s], 2 * C::GROUP);
+        constexpr uint32_t BOTH = 2 * C::GROUP;         // one group of both CTAs
+        for (int s = 0; s < C::NQ; ++s) mbar_init(&m->full_q[s], 1);
+        for (int s = 0; s < C::NKS; ++s) {
+            mbar_init(&m->full_ks[s], 1);
+            mbar_init(&m->snap_ready[s], BOTH);
         }
-        for (int s = 0; s < C::NDONE; ++s) {
-            mbar_init(&m->kv_done[s], 1);
+        for (int s = 0; s < C::NKD; ++s) mbar_init(&m->full_kd[s], 1);
+        for (int s = 0; s < C::NV; ++s) mbar_init(&m->full_v[s], 1);
+        for (int s = 0; s < C::NF; ++s) {
+            mbar_init(&m->f1_done[s], 1);
             mbar_init(&m->o_done[s], 1);
+            mbar_init(&m->f1_free[s], 2 * BOTH);        // groups P and O
         }
-        mbar_init(&m->tail_kv, 1);
-        mbar_init(&m->tail_zeroed, 2 * C::GROUP);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&m->snap_ready[i], 2 * C::GROUP);
-            mbar_init(&m->o_free[i], 2 * C::GROUP);
-            mbar_init(&m->dkv_free[i], 2 * C::GROUP);
+        for (int s = 0; s < C::NDK; ++s) {
+            mbar_init(&m->dkv_done[s], 1);
+            mbar_init(&m->dkv_free[s], BOTH);
         }
-        for (int i = 0; i < C::NPB; ++i) mbar_init(&m->p_ready[i], 2 * C::GROUP);
+        for (int s = 0; s < C::NPB; ++s) mbar_init(&m->p_ready[s], BOTH);
+        mbar_init(&m->tail_v, 1);
+        mbar_init(&m->tail_zeroed, BOTH);
         mbar_init(&m->drain, 2);
+        mbar_init(&m->done0, 1);
+        mbar_arrive(&m->done0);
         mbar_init(&m->ss_bar[0], C::GROUP);
         mbar_init(&m->ss_bar[1], C::GROUP);
         m->abort_flag = 0;
@@ -213,6 +192,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         tma_prefetch_desc(&p.tmap_k64);
         tma_prefetch_desc(&p.tmap_k128);
         tma_prefetch_desc(&p.tmap_v128);
+        tma_prefetch_desc(&p.tmap_o32);
     }
     if (warp == 1) {
         tmem_alloc_pair(&m->tmem_base, C::TMEM_COLS);
@@ -228,22 +208,21 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         *abort_flag = 1;
         record_fault(DEV_TIMEOUT);
     };
-    auto kk_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_KK + (j % C::NKK) * C::KK_BYTES); };
-    auto qh_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_QH + (j % C::NQH) * C::QH_BYTES); };
-    auto kv_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_KV + (j % C::NKV) * C::KV_BYTES); };
+    auto q_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_Q + (j % C::NQ) * C::Q_BYTES); };
+    auto ks_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_KS + (j % C::NKS) * C::KS_BYTES); };
+    auto kd_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_KD + (j % C::NKD) * C::T_BYTES); };
+    auto v_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_V + (j % C::NV) * C::T_BYTES); };
+    auto p_addr = [&](int j) { return sbase + (uint32_t)(C::OFF_P + (j % C::NPB) * C::P_BYTES); };
     // Bounded warp-uniform wait.  A CTA-scope poll suffices: remote producers
     // order their shared-memory writes with a cluster-scope release fence before
     // arriving, and MMA commits and TMA loads complete the barriers directly.
     auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, tlimit)) != 0;
     };
-    // Signals to CTA 0.  CTA 0's own threads arrive locally.  CTA 1's threads
-    // publish their shared-memory writes (P, the state snapshot, zeroed value
-    // rows) with a release fence restricted to shared memory and a relaxed
-    // remote arrival; a full cluster-scope release would also wait for the
-    // thread's outstanding global stores.  Signals that only free a TMEM buffer
-    // (the tcgen05.ld has completed) publish nothing and use a plain relaxed
-    // arrival.
+    // Signals to CTA 0.  CTA 1's threads publish their shared-memory writes (P, the
+    // snapshot, zeroed value rows) with a release fence restricted to shared memory
+    // and a relaxed remote arrival; signals that only free a TMEM buffer publish
+    // nothing and use a plain relaxed arrival.
     auto arrive_leader = [&](uint64_t *bar) {
         if (cta == 0) {
             mbar_arrive(bar);
@@ -258,19 +237,24 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         else
             mbar_arrive_cluster_relaxed(cluster_addr(bar, 0));
     };
+    // Rows [nv, 128) of a 128-row value tile set to zero by one epilogue group (128 threads).
+    auto zero_rows = [&](uint32_t tile, int nv, int gtid) {
+        for (uint32_t a = tile + (uint32_t)nv * 128 + (uint32_t)gtid * 16; a < tile + C::FBOX;
+             a += C::GROUP * 16)
+            st_shared_v4(a, 0u, 0u, 0u, 0u);
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
-        // One thread polls the three rings and refills whichever slot the MMAs have
+        // One thread polls the four rings and refills whichever slot its reader has
         // released.  CTA 0 expects the bytes of both CTAs on its full barrier; CTA 1's
-        // loads complete CTA 0's barrier directly.  The KV tiles of a partial last
-        // block are the exception: CTA 1 loads them against its own tail barrier, so
-        // that its group P can zero the value rows past the sequence end once they
-        // have landed, and CTA 0 expects only its own bytes for that block.
+        // loads complete CTA 0's barrier directly.  The value tile of a partial last
+        // block is the exception: CTA 1 loads it against its own tail barrier, so that
+        // its group KV can zero the rows past the sequence end once they have landed.
         if (lane == 0) {
             const int col = h * C::D;
             const int own_rows = 64 * (int)cta, own_cols = col + 64 * (int)cta;
-            int jk = 0, jq = 0, jv = 0;
+            int jq = 0, js = 0, jd = 0, jv = 0;
             // slot of block j free: block j - depth has released it
             auto freed = [&](uint64_t *ring, int nring, int j, int depth) {
                 const int x = j - depth;
@@ -278,30 +262,60 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             };
             uint64_t t0 = globaltimer_ns();
             uint32_t polls = 0;
-            while (jk < nb || jq < nb || jv < nb) {
+            while (jq < nb || js < nb || jd < nb || jv < nb) {
                 bool progressed = false;
-                if (jk < nb && freed(m->s_full, C::NS, jk, C::NKK)) {
-                    uint64_t *fb = &m->full_kk[jk % C::NKK];
-                    const uint32_t dst = kk_addr(jk);
-                    const int row = seq_start + jk * C::BETA + own_rows;
+                if (jd < nb && freed(m->dkv_done, C::NDK, jd, C::NKD)) {
+                    uint64_t *fb = &m->full_kd[jd % C::NKD];
+                    const uint32_t dst = kd_addr(jd);
+                    const int row = seq_start + jd * C::BETA;
                     if (cta == 0) {
-                        mbar_arrive_expect_tx(fb, (uint32_t)(2 * C::KK_BYTES));
+                        mbar_arrive_expect_tx(fb, (uint32_t)(2 * C::T_BYTES));
+                        tma_load_2d(dst, &p.tmap_k128, own_cols, row, fb);
+                    } else {
+                        tma_load_2d_pairbar(dst, &p.tmap_k128, own_cols, row, cluster_addr(fb, 0));
+                    }
+                    ++jd;
+                    progressed = true;
+                }
+                if (jv < nb && freed(m->o_done, C::NF, jv, C::NV)) {
+                    uint64_t *fb = &m->full_v[jv % C::NV];
+                    const uint32_t dst = v_addr(jv);
+                    const int row = seq_start + jv * C::BETA;
+                    const bool last_partial = tail && jv == nb - 1;
+                    if (cta == 0) {
+                        mbar_arrive_expect_tx(fb, (uint32_t)((last_partial ? 1 : 2) * C::T_BYTES));
+                        tma_load_2d(dst, &p.tmap_v128, own_cols, row, fb);
+                    } else if (last_partial) {
+                        mbar_arrive_expect_tx(&m->tail_v, (uint32_t)C::T_BYTES);
+                        tma_load_2d(dst, &p.tmap_v128, own_cols, row, &m->tail_v);
+                    } else {
+                        tma_load_2d_pairbar(dst, &p.tmap_v128, own_cols, row, cluster_addr(fb, 0));
+                    }
+                    ++jv;
+                    progressed = true;
+                }
+                if (js < nb && freed(m->f1_done, C::NF, js, C::NKS)) {
+                    uint64_t *fb = &m->full_ks[js % C::NKS];
+                    const uint32_t dst = ks_addr(js);
+                    const int row = seq_start + js * C::BETA + own_rows;
+                    if (cta == 0) {
+                        mbar_arrive_expect_tx(fb, (uint32_t)(4 * C::HBOX));
                         tma_load_2d(dst, &p.tmap_k64, col, row, fb);
-                        tma_load_2d(dst + C::HBOX, &p.tmap_k64, col + 64, row, fb);
+                        tma_load_2d(dst + C::FBOX, &p.tmap_k64, col + 64, row, fb);
                     } else {
                         const uint32_t fr = cluster_addr(fb, 0);
                         tma_load_2d_pairbar(dst, &p.tmap_k64, col, row, fr);
-                        tma_load_2d_pairbar(dst + C::HBOX, &p.tmap_k64, col + 64, row, fr);
+                        tma_load_2d_pairbar(dst + C::FBOX, &p.tmap_k64, col + 64, row, fr);
                     }
-                    ++jk;
+                    ++js;
                     progressed = true;
                 }
-                if (jq < nb && freed(m->o_done, C::NDONE, jq, C::NQH)) {
-                    uint64_t *fb = &m->full_qh[jq % C::NQH];
-                    const uint32_t dst = qh_addr(jq);
+                if (jq < nb && freed(m->f1_done, C::NF, jq, C::NQ)) {
+                    uint64_t *fb = &m->full_q[jq % C::NQ];
+                    const uint32_t dst = q_addr(jq);
                     const int row = seq_start + jq * C::BETA + own_rows;
                     if (cta == 0) {
-                        mbar_arrive_expect_tx(fb, (uint32_t)(2 * C::QH_BYTES));
+                        mbar_arrive_expect_tx(fb, (uint32_t)(2 * C::Q_BYTES));
                         tma_load_2d(dst, &p.tmap_q64, col, row, fb);
                         tma_load_2d(dst + C::HBOX, &p.tmap_q64, col + 64, row, fb);
                     } else {
@@ -310,28 +324,6 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                         tma_load_2d_pairbar(dst + C::HBOX, &p.tmap_q64, col + 64, row, fr);
                     }
                     ++jq;
-                    progressed = true;
-                }
-                if (jv < nb && freed(m->kv_done, C::NDONE, jv, C::NKV) &&
-                    freed(m->o_done, C::NDONE, jv, C::NKV)) {
-                    uint64_t *fb = &m->full_kv[jv % C::NKV];
-                    const uint32_t dst = kv_addr(jv);
-                    const int row = seq_start + jv * C::BETA;
-                    const bool last_partial = tail && jv == nb - 1;
-                    if (cta == 0) {
-                        mbar_arrive_expect_tx(fb, (uint32_t)((last_partial ? 1 : 2) * C::KV_BYTES));
-                        tma_load_2d(dst, &p.tmap_k128, own_cols, row, fb);
-                        tma_load_2d(dst + C::KV_OFF_VC, &p.tmap_v128, own_cols, row, fb);
-                    } else if (last_partial) {
-                        mbar_arrive_expect_tx(&m->tail_kv, (uint32_t)C::KV_BYTES);
-                        tma_load_2d(dst, &p.tmap_k128, own_cols, row, &m->tail_kv);
-                        tma_load_2d(dst + C::KV_OFF_VC, &p.tmap_v128, own_cols, row, &m->tail_kv);
-                    } else {
-                        const uint32_t fr = cluster_addr(fb, 0);
-                        tma_load_2d_pairbar(dst, &p.tmap_k128, own_cols, row, fr);
-                        tma_load_2d_pairbar(dst + C::KV_OFF_VC, &p.tmap_v128, own_cols, row, fr);
-                    }
-                    ++jv;
                     progressed = true;
                 }
                 if (progressed) {
@@ -349,141 +341,119 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             // exits.  CTA 1's loads are tracked by CTA 0's barriers; on the normal path
             // every one of them was consumed by an MMA, and after an abort the CTAs
             // wait out any load still in flight before they exit.
+            const uint64_t lim = tlimit < 10000000ull ? tlimit : 10000000ull;
             if (cta == 0) {
-                const uint64_t lim = tlimit < 10000000ull ? tlimit : 10000000ull;
-                for (int j = (jk > C::NKK ? jk - C::NKK : 0); j < jk; ++j)
-                    mbar_wait(&m->full_kk[j % C::NKK], (uint32_t)((j / C::NKK) & 1), nullptr, lim);
-                for (int j = (jq > C::NQH ? jq - C::NQH : 0); j < jq; ++j)
-                    mbar_wait(&m->full_qh[j % C::NQH], (uint32_t)((j / C::NQH) & 1), nullptr, lim);
-                for (int j = (jv > C::NKV ? jv - C::NKV : 0); j < jv; ++j)
-                    mbar_wait(&m->full_kv[j % C::NKV], (uint32_t)((j / C::NKV) & 1), nullptr, lim);
+                for (int j = (jq > C::NQ ? jq - C::NQ : 0); j < jq; ++j)
+                    mbar_wait(&m->full_q[j % C::NQ], (uint32_t)((j / C::NQ) & 1), nullptr, lim);
+                for (int j = (js > C::NKS ? js - C::NKS : 0); j < js; ++j)
+                    mbar_wait(&m->full_ks[j % C::NKS], (uint32_t)((j / C::NKS) & 1), nullptr, lim);
+                for (int j = (jd > C::NKD ? jd - C::NKD : 0); j < jd; ++j)
+                    mbar_wait(&m->full_kd[j % C::NKD], (uint32_t)((j / C::NKD) & 1), nullptr, lim);
+                for (int j = (jv > C::NV ? jv - C::NV : 0); j < jv; ++j)
+                    mbar_wait(&m->full_v[j % C::NV], (uint32_t)((j / C::NV) & 1), nullptr, lim);
             } else if (tail && jv == nb) {
-                mbar_wait(&m->tail_kv, 0u, nullptr, tlimit < 10000000ull ? tlimit : 10000000ull);
+                mbar_wait(&m->tail_v, 0u, nullptr, lim);
             }
         }
         __syncwarp();
-    } else if (warp == 1 && cta == 0) {
-        // ------------------------------------------------------------ issuer A (CTA 0): S, dKV
-        // One thread issues tcgen05.mma at well under the tensor pipe's rate for these
-        // M = 128 (64 rows per CTA), N = 128 paired MMAs, so the work is split between two
-        // issuing warps: A issues the products that depend only on loads (S and dKV), B
-        // those that wait on the epilogue warps (the inter-block term and P V).  A commit
-        // covers the MMAs of its own thread only.
-        auto stage_in = [&](int j) -> bool {  // S_j = Q_j K_j^T
-            if (!wwait(&m->full_kk[j % C::NKK], (uint32_t)((j / C::NKK) & 1)) ||
-                !wwait(&m->full_qh[j % C::NQH], (uint32_t)((j / C::NQH) & 1)))
-                return false;
-            // S buffer j % NS was last read by group P for block j - NS
-            if (j >= C::NS && !wwait(&m->s_free[j % C::NS], (uint32_t)(((j - C::NS) / C::NS) & 1)))
-                return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t qd = desc_kmajor_sw128(qh_addr(j));
-                const uint64_t kd = desc_kmajor_sw128(kk_addr(j));
-#pragma unroll
-                for (int ks = 0; ks < C::D / 16; ++ks) {
-                    const uint32_t off = (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32);
-                    mma_bf16_ss_pair(tmem + C::TM_S + 64 * (j % C::NS), desc_add(qd, off),
-                                     desc_add(kd, off), C::ID_S, ks > 0 ? 1u : 0u);
-                }
-                mma_commit_pair_both(&m->s_full[j % C::NS]);
-            }
-            __syncwarp();
-            return true;
-        };
-        // Per block b: dKV_b^T = V_b^T K_b, then S_{b+SAHEAD} (look-ahead, so that group P
-        // has SAHEAD blocks' time to form P from it).  dKV_b goes first: the snapshot of
-        // KV_{<b+1} that issuer B waits for is derived from it.
-        bool ok = true;
-        for (int j = 0; ok && j < C::SAHEAD && j < nb; ++j) ok = stage_in(j);
-        for (int b = 0; ok && b < nb; ++b) {
-            const uint32_t kva = kv_addr(b);
-            // a partial last block: group P zeroes the value rows past the sequence end
-            // before dKV_b may read them
-            const bool zero_tail = tail && b == nb - 1;
-            if ((zero_tail && !wwait(&m->tail_zeroed, 0u)) ||
-                !wwait(&m->full_kv[b % C::NKV], (uint32_t)((b / C::NKV) & 1)) ||
-                (b >= 2 && !wwait(&m->dkv_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t vd = desc_mnmajor_sw128(kva + C::KV_OFF_VC, C::FBOX);
-                const uint64_t kd = desc_mnmajor_sw128(kva, C::FBOX);
+    } else if (warp == 1 || warp == C::WARP_D) {
+        if (cta == 0) {
+            // -------------------------------------------------------- issuers (CTA 0)
+            // Lane 0 alone waits and issues.  Before each product it probes every barrier
+            // the product needs at once (one round trip to the barriers for all of them)
+            // and falls back to a bounded wait on each only when one is not complete yet.
+            // Unused slots name done0, whose phase 0 is always complete.
+            auto ready = [&](uint64_t *b0, uint32_t p0, uint64_t *b1, uint32_t p1, uint64_t *b2,
+                             uint32_t p2, uint64_t *b3, uint32_t p3) -> bool {
+                if (mbar_test4(b0, p0, b1, p1, b2, p2, b3, p3)) return true;
+                return mbar_wait(b0, p0, abort_flag, tlimit) && mbar_wait(b1, p1, abort_flag, tlimit) &&
+                       mbar_wait(b2, p2, abort_flag, tlimit) && mbar_wait(b3, p3, abort_flag, tlimit);
+            };
+            uint64_t *const any = &m->done0;
+            // dKV_j^T = V_j^T K_j into dKV buffer j % NDK.  Waits: key dims and values of
+            // block j landed (their next phases need dKV_j itself); dKV_{j-NDK} loaded by
+            // group KV (the next phase needs dKV_j); for a partial last block, the value
+            // rows past the sequence end zeroed.
+            auto dkv = [&](int j) -> bool {
+                const bool last_tail = tail && j == nb - 1;
+                if (!ready(&m->full_kd[j % C::NKD], (uint32_t)((j / C::NKD) & 1),
+                           &m->full_v[j % C::NV], (uint32_t)((j / C::NV) & 1),
+                           j >= C::NDK ? &m->dkv_free[j % C::NDK] : any,
+                           j >= C::NDK ? (uint32_t)(((j - C::NDK) / C::NDK) & 1) : 0u,
+                           last_tail ? &m->tail_zeroed : any, 0u))
+                    return false;
+                tc_fence_after();
+                const uint64_t vd = desc_mnmajor_sw128(v_addr(j), C::FBOX);
+                const uint64_t kd = desc_mnmajor_sw128(kd_addr(j), C::FBOX);
 #pragma unroll
                 for (int ks = 0; ks < C::BETA / 16; ++ks)
-                    mma_bf16_ss_pair(tmem + C::TM_DKV + 64 * (b & 1), desc_add(vd, ks * 2048),
+                    mma_bf16_ss_pair(tmem + C::TM_DKV + 64 * (j % C::NDK), desc_add(vd, ks * 2048),
                                      desc_add(kd, ks * 2048), C::ID_KV, ks > 0 ? 1u : 0u);
-                mma_commit_pair_both(&m->kv_done[b % C::NDONE]);
-            }
-            __syncwarp();
-            if (b + C::SAHEAD < nb && !stage_in(b + C::SAHEAD)) {
-                ok = false;
-                break;
-            }
-        }
-        if (!ok) fail();
-        if (lane == 0) {  // every MMA of both issuers has finished before TMEM is freed
-            mma_commit_pair(smem_u32(&m->drain));
-            mbar_wait(&m->drain, 0u, nullptr, tlimit);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // CTA 1's warp 1 only takes part in the TMEM allocation.
-    } else if (warp == C::WARP_B) {
-        if (cta == 0) {
-            // -------------------------------------------------------- issuer B (CTA 0): O
-            // Per block b: O_b = Q_b snap(KV_{<b}), then O_b += P_b V_b.
-            bool ok = true;
-            for (int b = 0; ok && b < nb; ++b) {
-                const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
-                // The query tile of block b must have landed: nothing else that this thread
-                // waits for implies it (S_b was issued by the other thread, and the
-                // snapshot does not depend on it).  Checked for every block, in order.
-                if ((b >= 2 && !wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1))) ||
-                    !wwait(&m->full_qh[b % C::NQH], (uint32_t)((b / C::NQH) & 1))) {
-                    ok = false;
-                    break;
-                }
-                if (b >= u0) {
-                    // snapshot b is the (b - u0)/2-th use of buffer b % 2
-                    if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint64_t qd = desc_kmajor_sw128(qh_addr(b));
-                        const uint64_t sd = desc_kmajor_sw128(sbase + C::OFF_SNAP + (b & 1) * C::SNAP_BYTES);
+                mma_commit_pair_both(&m->dkv_done[j % C::NDK]);
+                return true;
+            };
+            // F1_j = [S_j | O_j] = Q_j [K_j ; snap_j]^T into region j % NF.  Waits: query
+            // and key rows landed and snapshot j written (their next phases need F1_j);
+            // region j % NF loaded by groups P and O for block j - NF (the next phase needs
+            // F1_j).
+            auto f1 = [&](int j) -> bool {
+                if (!ready(&m->full_q[j % C::NQ], (uint32_t)((j / C::NQ) & 1),
+                           &m->full_ks[j % C::NKS], (uint32_t)((j / C::NKS) & 1),
+                           &m->snap_ready[j % C::NKS], (uint32_t)((j / C::NKS) & 1),
+                           j >= C::NF ? &m->f1_free[j % C::NF] : any,
+                           j >= C::NF ? (uint32_t)(((j - C::NF) / C::NF) & 1) : 0u))
+                    return false;
+                tc_fence_after();
+                const uint64_t qd = desc_kmajor_sw128(q_addr(j));
+                const uint64_t bd = desc_kmajor_sw128(ks_addr(j));
 #pragma unroll
-                        for (int ks = 0; ks < C::D / 16; ++ks) {
-                            const uint32_t off = (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32);
-                            mma_bf16_ss_pair(dO, desc_add(qd, off), desc_add(sd, off), C::ID_QKV,
-                                             ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < C::D / 16; ++ks)
+                    mma_bf16_ss_pair(tmem + C::TM_F1 + 128 * (j % C::NF),
+                                     desc_add(qd, (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32)),
+                                     desc_add(bd, (uint32_t)((ks >> 2) * C::FBOX + (ks & 3) * 32)),
+                                     C::ID_F1, ks > 0 ? 1u : 0u);
+                mma_commit_pair_both(&m->f1_done[j % C::NF]);
+                return true;
+            };
+            // O_j += P_j V_j onto the O half of region j % NF, issued after F1_j by this
+            // thread.  Waits: P_j stored (the next phase needs o_done(j)).  The value tile
+            // landed: the dKV issuer waited for it before dKV_j, whose completion group KV
+            // saw before the snapshot F1_{j+1} waited for; and the next load into its slot
+            // needs o_done(j).  It is waited for here all the same (one probe).
+            auto pv = [&](int j) -> bool {
+                if (!ready(&m->p_ready[j % C::NPB], (uint32_t)((j / C::NPB) & 1),
+                           &m->full_v[j % C::NV], (uint32_t)((j / C::NV) & 1), any, 0u, any, 0u))
+                    return false;
+                tc_fence_after();
+                const uint64_t pd = desc_kmajor_sw128(p_addr(j));
+                const uint64_t vd = desc_mnmajor_sw128(v_addr(j), C::FBOX);
+#pragma unroll
+                for (int ks = 0; ks < C::BETA / 16; ++ks)
+                    mma_bf16_ss_pair(tmem + C::TM_F1 + 128 * (j % C::NF) + 64,
+                                     desc_add(pd, (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32)),
+                                     desc_add(vd, ks * 2048), C::ID_PV, 1u);
+                mma_commit_pair_both(&m->o_done[j % C::NF]);
+                return true;
+            };
+            bool ok = true;
+            if (lane == 0) {
+                if (warp == C::WARP_D) {
+                    for (int j = 0; ok && j < nb; ++j) ok = dkv(j);
+                } else {
+                    if (nb > 0) ok = f1(0);
+                    for (int b = 0; ok && b < nb; ++b) {
+                        if (b + 1 < nb && !f1(b + 1)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!pv(b)) {
+                            ok = false;
+                            break;
                         }
                     }
-                    __syncwarp();
                 }
-                if (!wwait(&m->p_ready[b % C::NPB], (uint32_t)((b / C::NPB) & 1)) ||
-                    !wwait(&m->full_kv[b % C::NKV], (uint32_t)((b / C::NKV) & 1))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t pd = desc_kmajor_sw128(sbase + C::OFF_P + (b % C::NPB) * C::P_BYTES);
-                    const uint64_t vd = desc_mnmajor_sw128(kv_addr(b) + C::KV_OFF_VC, C::FBOX);
-#pragma unroll
-                    for (int ks = 0; ks < C::BETA / 16; ++ks)
-                        mma_bf16_ss_pair(dO, desc_add(pd, (uint32_t)((ks >> 2) * C::HBOX + (ks & 3) * 32)),
-                                         desc_add(vd, ks * 2048), C::ID_PV, (b >= u0 || ks > 0) ? 1u : 0u);
-                    mma_commit_pair_both(&m->o_done[b % C::NDONE]);
-                }
-                __syncwarp();
-            }
-            if (!ok) fail();
-            if (lane == 0) {
+                if (!ok) fail();
+                // every MMA of both issuers has finished before TMEM is freed
                 mma_commit_pair(smem_u32(&m->drain));
                 mbar_wait(&m->drain, 0u, nullptr, tlimit);
             }
@@ -496,21 +466,22 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         const int r = 32 * (q & 1) + lane;     // own query row (0..63)
         const int kh = q >> 1;                 // key half held by this lane
         const int R = 64 * (int)cta + r;       // row within the block
-        const uint32_t sP = sbase + C::OFF_P;
         bool ok = true;
-        for (int b = 0; b < nb; ++b) {
-            if (!wwait(&m->s_full[b % C::NS], (uint32_t)((b / C::NS) & 1))) {
+        for (int j = 0; j < nb; ++j) {
+            // f1_done[j % NF] phase j / NF; the next phase (F1_{j+NF}) needs f1_free,
+            // which needs this group's load below
+            if (!wwait(&m->f1_done[j % C::NF], (uint32_t)((j / C::NF) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t s0[32], s1[32];
-            const uint32_t tS = tmem + C::TM_S + 64 * (b % C::NS) + lane_base;
+            const uint32_t tS = tmem + C::TM_F1 + 128 * (j % C::NF) + lane_base;
             tmem_ld32(tS, s0);
             tmem_ld32(tS + 32, s1);
             tmem_ld_wait();
             tc_fence_before();
-            arrive_leader_free(&m->s_free[b % C::NS]);
+            arrive_leader_free(&m->f1_free[j % C::NF]);
             uint32_t w[32];
 #pragma unroll
             for (int u = 0; u < 32; ++u) {
@@ -520,107 +491,135 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                 const float x1 = c0 + 1 <= R ? __uint_as_float(s[1]) : 0.f;
                 w[u] = pack_bf16x2(x0, x1);
             }
-            // P buffer b % NPB was last read by O_{b-NPB} += P V; that must be complete
-            const int pb = b - C::NPB;
-            if (pb >= 0 && !wwait(&m->o_done[pb % C::NDONE], (uint32_t)((pb / C::NDONE) & 1))) {
+            // The P buffer was last read by P_{j-NPB} V: o_done phase (j - NPB) / NF.  Its
+            // next phase (P V of block j - NPB + NF) needs P of a later block.
+            const int pb = j - C::NPB;
+            if (pb >= 0 && !wwait(&m->o_done[pb % C::NF], (uint32_t)((pb / C::NF) & 1))) {
                 ok = false;
                 break;
             }
+            const uint32_t sP = p_addr(j);
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-                st_shared_v4(sP + (b % C::NPB) * C::P_BYTES + kh * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4), w[4 * t],
+                st_shared_v4(sP + kh * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4), w[4 * t],
                              w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
-            // V rows past the sequence end must not enter dKV^T: zero them in this CTA's
-            // slice once its KV tiles of the block have landed.
-            const int nv = min(C::BETA, seq_len - b * C::BETA);
-            if (nv < C::BETA) {
-                const bool landed = cta == 0 ? wwait(&m->full_kv[b % C::NKV], (uint32_t)((b / C::NKV) & 1))
-                                             : wwait(&m->tail_kv, 0u);
-                if (!landed) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t v0 = kv_addr(b) + C::KV_OFF_VC;
-                for (uint32_t a = v0 + nv * 128 + (threadIdx.x - 64) * 16; a < v0 + C::FBOX;
-                     a += C::GROUP * 16)
-                    st_shared_v4(a, 0u, 0u, 0u, 0u);
-                fence_proxy_async_smem();
-                arrive_leader(&m->tail_zeroed);
-            }
             fence_proxy_async_smem();
-            tc_fence_before();
-            arrive_leader(&m->p_ready[b % C::NPB]);
+            arrive_leader(&m->p_ready[j % C::NPB]);
         }
         if (!ok) fail();
-    } else {
-        // ------------------------------------------------------------ group O (both CTAs)
+    } else if (warp < 10) {
+        // ------------------------------------------------------------ group KV (both CTAs)
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int r = 32 * (q & 1) + lane;     // own output row / own value column j
-        const int half = q >> 1;               // column half (O) / dim half (state)
+        const int r = 32 * (q & 1) + lane;     // own value column j (0..63)
+        const int half = q >> 1;               // dim half of the state
         float kv[64];                          // KV^T[64 c + r][64 half .. 64 half + 63]
 #pragma unroll
         for (int t = 0; t < 64; ++t) kv[t] = 0.f;
         bool ok = true;
-        // snapshot u of the state into buffer u % 2 (own 64 rows of KV^T, bf16, swizzled)
+        // snapshot u (the state before block u) into the snapshot rows of key-row slot u % NKS
         auto write_snap = [&](int u) {
-            const uint32_t sSnap = sbase + C::OFF_SNAP + (u & 1) * C::SNAP_BYTES;
+            const uint32_t dst = ks_addr(u) + half * C::FBOX + C::HBOX;
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-                st_shared_v4(sSnap + half * C::HBOX + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4),
+                st_shared_v4(dst + r * 128 + ((uint32_t)(t ^ (r & 7)) << 4),
                              pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
                              pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
                              pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
                              pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
             fence_proxy_async_smem();
-            arrive_leader(&m->snap_ready[u & 1]);
+            arrive_leader(&m->snap_ready[u % C::NKS]);
         };
-        if (p.state_in != nullptr) {  // KV^T[j][i] starts at the initial state X[i][j]
+        // The value rows past the end of a partial last block must not enter dKV^T (nor
+        // P V): zero them in this CTA's value tile once it has landed.  Done one block
+        // before that block's dKV (or first, for a one-block sequence), so that the dKV
+        // issuer never waits for work that depends on products it has not issued.  CTA
+        // 0's wait is exact: the slot's previous load (block nb - 1 - NV) fed
+        // dKV_{nb-1-NV}, which this group has already seen complete.
+        auto zero_tail = [&]() -> bool {
+            const int b = nb - 1;
+            const bool landed = cta == 0 ? wwait(&m->full_v[b % C::NV], (uint32_t)((b / C::NV) & 1))
+                                         : wwait(&m->tail_v, 0u);
+            if (!landed) return false;
+            zero_rows(v_addr(b), seq_len - b * C::BETA, (int)threadIdx.x - 64 - C::GROUP);
+            fence_proxy_async_smem();
+            arrive_leader(&m->tail_zeroed);
+            return true;
+        };
+        if (p.state_in != nullptr && (nb > 0 || p.state != nullptr)) {
+            // KV^T[j][i] starts at the initial state X[i][j]
             const float *src = p.state_in + ((size_t)sid * p.H + h) * C::D * C::D + 64 * (int)cta + r;
 #pragma unroll
             for (int t = 0; t < 64; ++t) kv[t] = src[(size_t)(64 * half + t) * C::D];
-            write_snap(0);
         }
-        for (int b = 0; b < nb; ++b) {
-            // (1) state: KV^T += dKV_b^T, then the bf16 snapshot for O_{b+1} += Q_{b+1} KV
-            if (!wwait(&m->kv_done[b % C::NDONE], (uint32_t)((b / C::NDONE) & 1))) {
+        if (nb > 0) {
+            write_snap(0);
+            if (tail && nb == 1) ok = zero_tail();
+        }
+        for (int b = 0; ok && b < nb; ++b) {
+            if (tail && nb >= 2 && b == nb - 2 && !zero_tail()) {
+                ok = false;
+                break;
+            }
+            // dkv_done[b % NDK] phase b / NDK; the next phase needs dkv_free from below
+            if (!wwait(&m->dkv_done[b % C::NDK], (uint32_t)((b / C::NDK) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            const uint32_t tK = tmem + C::TM_DKV + 64 * (b % C::NDK) + lane_base;
             {
-                uint32_t a[32], c[32];
-                const uint32_t tK = tmem + C::TM_DKV + 64 * (b & 1) + lane_base;
+                uint32_t a[32];
                 tmem_ld32(tK, a);
-                tmem_ld32(tK + 32, c);
                 tmem_ld_wait();
-                tc_fence_before();
-                arrive_leader_free(&m->dkv_free[b & 1]);
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    kv[t] += __uint_as_float(a[t]);
-                    kv[32 + t] += __uint_as_float(c[t]);
-                }
+                for (int t = 0; t < 32; ++t) kv[t] += __uint_as_float(a[t]);
+                tmem_ld32(tK + 32, a);
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 32; ++t) kv[32 + t] += __uint_as_float(a[t]);
             }
+            tc_fence_before();
+            arrive_leader_free(&m->dkv_free[b % C::NDK]);
             if (b + 1 < nb) {
-                // Snapshot b + 1 goes to buffer (b+1) & 1, last read by O_{b-1} = Q_{b-1}
-                // snap_{b-1}, complete since o_done(b-1), which this group waited for in
-                // the previous block.
+                // slot (b+1) % NKS was last read by F1_{b+1-NKS}: f1_done phase
+                // (b+1-NKS) / NF; its next phase needs snapshot b+1-NKS+NF, written later
+                const int x = b + 1 - C::NKS;
+                if (x >= 0 && !wwait(&m->f1_done[x % C::NF], (uint32_t)((x / C::NF) & 1))) {
+                    ok = false;
+                    break;
+                }
                 write_snap(b + 1);
             }
-            // (2) output block b
-            if (!wwait(&m->o_done[b % C::NDONE], (uint32_t)((b / C::NDONE) & 1))) {
+        }
+        if (ok && p.state != nullptr) {  // final state (fp32), state[i][j] = KV^T[j][i]
+            float *dst = p.state + ((size_t)sid * p.H + h) * C::D * C::D + 64 * (int)cta + r;
+#pragma unroll
+            for (int t = 0; t < 64; ++t) dst[(size_t)(64 * half + t) * C::D] = kv[t];
+        }
+        if (!ok) fail();
+    } else if (warp < C::WARP_D) {
+        // ------------------------------------------------------------ group O (both CTAs)
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int r = 32 * (q & 1) + lane;     // own output row
+        const int half = q >> 1;               // column half
+        bool ok = true;
+        for (int b = 0; b < nb; ++b) {
+            // o_done[b % NF] phase b / NF; the next phase (P V of block b + NF) needs
+            // F1_{b+NF}, which needs f1_free from the load below
+            if (!wwait(&m->o_done[b % C::NF], (uint32_t)((b / C::NF) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t a[32], c[32];
-            const uint32_t tO = tmem + C::TM_O + 64 * (b & 1) + lane_base;
+            const uint32_t tO = tmem + C::TM_F1 + 128 * (b % C::NF) + 64 + lane_base;
             tmem_ld32(tO, a);
             tmem_ld32(tO + 32, c);
             tmem_ld_wait();
             tc_fence_before();
-            arrive_leader_free(&m->o_free[b & 1]);
+            arrive_leader_free(&m->f1_free[b % C::NF]);
             float scale = 1.0f;
             if (p.rmsnorm) {
                 float ss = 0.f;
@@ -630,7 +629,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                     ss = fmaf(x, x, ss);
                     ss = fmaf(y, y, ss);
                 }
-                // exchange with the lane holding the other column half (bounded wait)
+                // exchange with warp q ^ 2, which holds the other column half of the row
                 m->ss_x[b & 1][half][r] = ss;
                 mbar_arrive(&m->ss_bar[b & 1]);
                 if (!__all_sync(0xffffffffu, mbar_wait(&m->ss_bar[b & 1], (uint32_t)((b >> 1) & 1),
@@ -644,7 +643,32 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             }
             const int nv = min(C::BETA, seq_len - b * C::BETA);
             const int R = 64 * (int)cta + r;
-            if (R < nv) {
+            const int R0 = 64 * (int)cta + 32 * (q & 1);     // first row of this warp's box
+            if (R0 + 32 <= nv) {
+                // the whole box lies inside the sequence: stage it (128-byte swizzle) and let
+                // one lane issue a TMA store.  Register-to-global stores would wait in this
+                // SM's memory pipe while HBM is saturated and hold up the MMA issue behind them.
+                const uint32_t stage = sbase + C::OFF_OST + q * C::OST_BYTES;
+                if (lane == 0) bulk_wait_read_all();   // the previous box has been read
+                __syncwarp();
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const uint32_t *src = t < 4 ? &a[8 * t] : &c[8 * (t - 4)];
+                    st_shared_v4(stage + lane * 128 + ((uint32_t)(t ^ (lane & 7)) << 4),
+                                 pack_bf16x2(__uint_as_float(src[0]) * scale, __uint_as_float(src[1]) * scale),
+                                 pack_bf16x2(__uint_as_float(src[2]) * scale, __uint_as_float(src[3]) * scale),
+                                 pack_bf16x2(__uint_as_float(src[4]) * scale, __uint_as_float(src[5]) * scale),
+                                 pack_bf16x2(__uint_as_float(src[6]) * scale, __uint_as_float(src[7]) * scale));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&p.tmap_o32, stage, h * C::D + 64 * half, seq_start + b * C::BETA + R0);
+                    bulk_commit_group();
+                }
+                __syncwarp();
+            } else if (R < nv) {
+                // the partial last block: plain stores of the rows inside the sequence
                 uint4 *dst = reinterpret_cast<uint4 *>(
                     p.o + ((size_t)(seq_start + b * C::BETA + R) * p.H + h) * C::D + 64 * half);
 #pragma unroll
@@ -658,11 +682,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                 }
             }
         }
-        if (ok && p.state != nullptr) {  // final state K^T V (fp32), state[i][j] = KV^T[j][i]
-            float *dst = p.state + ((size_t)sid * p.H + h) * C::D * C::D + 64 * (int)cta + r;
-#pragma unroll
-            for (int t = 0; t < 64; ++t) dst[(size_t)(64 * half + t) * C::D] = kv[t];
-        }
+        if (lane == 0) bulk_wait_all();   // every O box stored before the CTA leaves
+        __syncwarp();
         if (!ok) fail();
     }
 

@@ -26,19 +26,17 @@ from . import api
 
 
 def all_gather_states(local: torch.Tensor, group=None) -> torch.Tensor:
-    """[R, *local.shape]: every rank's local state, in rank order, on every rank."""
+    """[R, *local.shape]: every rank's local state, in rank order, on every rank.
+
+    One ``all_gather_into_tensor`` into a buffer that holds the R local states one after
+    the other along the first axis: the layout both NCCL and gloo accept, so that the CPU
+    tests run the same call as the GPU ranks."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    gathered = local.new_empty((world,) + tuple(local.shape))
-    if dist.get_backend(group) == "nccl":
-        dist.all_gather_into_tensor(gathered, local.contiguous(), group=group)
-    else:
-        parts = list(gathered.unbind(0))
-        dist.all_gather(parts, local.contiguous(), group=group)
-        for dst, src in zip(gathered.unbind(0), parts):
-            if dst.data_ptr() != src.data_ptr():
-                dst.copy_(src)
-    return gathered
+    local = local.contiguous()
+    flat = local.new_empty((world * local.shape[0],) + tuple(local.shape[1:]))
+    dist.all_gather_into_tensor(flat, local, group=group)
+    return flat.view((world,) + tuple(local.shape))
 
 
 def chunk_prefill(q, k, v, gathered, rank: int, *, beta: int = 128, cu_seqlens=None,

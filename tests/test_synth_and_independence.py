@@ -114,7 +114,8 @@ def test_native_sources_include_nothing_of_each_other():
 
 def test_bench_uses_the_oracle_only_for_the_cpu_timing():
     tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
-    allowed = {"time_oracle_prefill"}
+    # the only functions that may use the oracle: the CPU-baseline timings
+    allowed = {"time_oracle_prefill", "cpu_oracle_prefill", "cpu_oracle_quadratic", "decode_cpu_baseline"}
     for fn in ast.walk(tree):
         if isinstance(fn, ast.FunctionDef):
             for node in ast.walk(fn):
@@ -135,3 +136,19 @@ def test_bench_uses_the_oracle_only_for_the_cpu_timing():
                for node in ast.walk(fn) if isinstance(node, ast.Call)
                and getattr(node.func, "id", None) == "time_oracle_prefill"}
     assert callers == {"cpu_baseline", "run_reference"}, callers
+
+    def callers_of(name):
+        return {fn.name for fn in ast.walk(tree) if isinstance(fn, ast.FunctionDef)
+                for node in ast.walk(fn) if isinstance(node, ast.Call)
+                and getattr(node.func, "id", None) == name}
+    # the per-config baselines run inside bench_configs only under its `cpu` switch, and the
+    # decode baseline only on rank 0 of a 1-GPU run
+    assert callers_of("cpu_oracle_prefill") == {"bench_configs"}
+    assert callers_of("cpu_oracle_quadratic") == {"bench_configs"}
+    assert callers_of("decode_cpu_baseline") == {"run_ours"}
+    cfg = next(fn for fn in ast.walk(tree) if isinstance(fn, ast.FunctionDef) and fn.name == "bench_configs")
+    for node in ast.walk(cfg):
+        if isinstance(node, ast.Call) and getattr(node.func, "id", "") in ("cpu_oracle_prefill", "cpu_oracle_quadratic"):
+            guarded = any(isinstance(i, ast.If) and isinstance(i.test, ast.Name) and i.test.id == "cpu"
+                          and any(c is node for c in ast.walk(i)) for i in ast.walk(cfg))
+            assert guarded, "a per-config CPU baseline outside the `if cpu:` switch"
