@@ -84,6 +84,9 @@ struct PairCfg {
     // A ring's slot of block x is tested free on the done barrier of block x, which
     // must not have been lapped (by block x + ring size) when the producer tests it.
     static_assert(NQ <= NF && NKS <= NF && NV <= NF && NKD <= NDK && NPB <= NF, "release rings");
+    // Group KV waits for the value tile of a partial last block one block before its dKV:
+    // the wait is exact only if the slot's previous load fed a dKV it has seen complete.
+    static_assert(NV >= 2, "value ring: group KV's tail wait");
     static constexpr int Q_BYTES = 2 * HBOX, KS_BYTES = 2 * FBOX, T_BYTES = FBOX;
     static constexpr int P_BYTES = 2 * HBOX;
     static constexpr int OST_BYTES = 32 * 128;          // one 32-row x 64-column O box

@@ -6,9 +6,11 @@ buffer, state snapshot and TMEM accumulator holds, and the mbarriers that order 
 Each agent is a generator that mirrors one role of the kernel, one step per wait,
 arrival, TMA issue, store or MMA issue, in the kernel's order:
 
-    producer0, producer1   warp 0 of CTA 0 / CTA 1 (the three TMA rings)
-    A, B                   the two MMA-issuing warps of CTA 0
-    P<c>.<w>, O<c>.<w>     warp w (0..3) of group P / group O in CTA c
+    producer0, producer1   warp 0 of CTA 0 / CTA 1 (the four TMA rings)
+    A                      CTA 0's issuer of F1 = Q [K ; snap]^T and P V
+    D                      CTA 0's issuer of dKV^T = V^T K
+    P<c>.<w>, KV<c>.<w>, O<c>.<w>
+                           warp w (0..3) of group P / KV / O in CTA c
 
 Asynchronous work is a pool of pending events that fire in random order, interleaved at
 random with the agents' steps: each TMA tile landing (its transaction bytes on its
@@ -25,13 +27,15 @@ Every schedule is checked for:
   * an MMA issued only on operands that hold the intended block's data, fully landed,
     with the value rows past the sequence end zeroed for the partial last block, and
     never overwriting an accumulator that a warp still has to load;
+  * the O accumulator loaded only after both of its products (F1, then P V) completed;
   * a TMEM load only of the intended block's accumulator, with all its MMAs complete;
   * no shared-memory write (TMA or store) to a buffer that an in-flight MMA reads;
   * the RMSNorm partial sums read only after their writer stored them, and never
     overwritten before the partner lane read them;
   * no deadlock, and nothing in flight once every agent has finished.
 
-Not modelled: the timeout / abort paths, TMEM allocation, the numerical content.
+Not modelled: the timeout / abort paths, TMEM allocation, the numerical content, the
+output's TMA store (its staging buffer is read by no MMA).
 """
 from __future__ import annotations
 
@@ -40,9 +44,8 @@ import random
 BETA = 128
 HBOX = 64 * 128          # one 64-row x 128-byte TMA tile
 FBOX = 128 * 128         # one 128-row x 128-byte TMA tile
-KK_BYTES = QH_BYTES = 2 * HBOX
-KV_BYTES = 2 * FBOX
-NDONE = 4                # ring of block-completion barriers (kv_done, o_done)
+NF = 3                   # F1 TMEM regions [S | O] (and the f1_done / o_done / f1_free rings)
+NDK = 2                  # dKV TMEM buffers (and the dkv_done / dkv_free rings)
 WARPS = 4                # warps per epilogue group
 
 
@@ -109,49 +112,47 @@ class PairModel:
     """One CTA pair working on one (sequence, head) of ``nb`` blocks.
 
     tail: the last block is partial.  init: the kernel starts from an initial state.
-    kk, qh, kv, pbufs, sahead: ring depths (LA_PAIR_KK_DEPTH, LA_PAIR_QH_DEPTH,
-    LA_PAIR_KV_DEPTH, LA_PAIR_P_BUFS, LA_PAIR_S_AHEAD).  ``mutations`` names deliberate
-    protocol mistakes, for checking that the model catches them.
+    nq, nks, nkd, nv, npb: ring depths (PairCfg::NQ, NKS, NKD, NV, NPB).  ``mutations``
+    names deliberate protocol mistakes, for checking that the model catches them.
     """
 
-    def __init__(self, nb, tail=False, init=False, rms=False, kk=2, qh=4, kv=2, pbufs=1,
-                 sahead=1, mutations=(), static_checks=True):
+    def __init__(self, nb, tail=False, init=False, rms=False, nq=2, nks=2, nkd=2, nv=3, npb=2,
+                 mutations=(), static_checks=True):
         self.nb, self.tail, self.init, self.rms = nb, tail and nb > 0, init, rms
-        self.NKK, self.NQH, self.NKV, self.NPB = kk, qh, kv, pbufs
-        self.SAHEAD, self.NS = sahead, sahead + 1
+        self.NQ, self.NKS, self.NKD, self.NV, self.NPB = nq, nks, nkd, nv, npb
         self.mut = frozenset(mutations)
-        if static_checks and not self.compiles(kk, qh, kv, pbufs, sahead):
-            raise ValueError("ring depths rejected by the kernel's static_asserts")
-        self.u0 = 0 if init else 1
+        if static_checks and not self.compiles(nq, nks, nkd, nv, npb):
+            raise ValueError("ring depths rejected by the kernel's static_assert")
         self.bars = [self._cta_bars(c) for c in (0, 1)]
         P_ids = [{("P", c, w) for w in range(WARPS)} for c in (0, 1)]
+        KV_ids = [{("KV", c, w) for w in range(WARPS)} for c in (0, 1)]
         O_ids = [{("O", c, w) for w in range(WARPS)} for c in (0, 1)]
-        self.KK = [[[Buf(f"KK{s}.{h}@{c}") for h in (0, 1)] for s in range(self.NKK)] for c in (0, 1)]
-        self.QH = [[[Buf(f"QH{s}.{h}@{c}") for h in (0, 1)] for s in range(self.NQH)] for c in (0, 1)]
-        self.KV = [[{"K": Buf(f"KV{s}.K@{c}"), "V": Buf(f"KV{s}.V@{c}")} for s in range(self.NKV)]
-                   for c in (0, 1)]
-        self.P = [[[Buf(f"P{s}.{w}@{c}") for w in range(WARPS)] for s in range(self.NPB)] for c in (0, 1)]
-        nsnap = 1 if "one_snapshot" in self.mut else 2
-        self.NSNAP = nsnap
-        self.SNAP = [[[Buf(f"SNAP{s}.{w}@{c}") for w in range(WARPS)] for s in range(nsnap)]
-                     for c in (0, 1)]
-        self.S = [[Buf(f"tmS{s}@{c}", P_ids[c]) for s in range(self.NS)] for c in (0, 1)]
-        self.O = [[Buf(f"tmO{s}@{c}", O_ids[c]) for s in range(2)] for c in (0, 1)]
-        self.DKV = [[Buf(f"tmDKV{s}@{c}", O_ids[c]) for s in range(2)] for c in (0, 1)]
+        self.Q = [[[Buf(f"Q{s}.{h}@{c}") for h in (0, 1)] for s in range(nq)] for c in (0, 1)]
+        # key-row slot: the TMA'd key rows (per dim half) and the snapshot rows (per KV warp)
+        self.KSK = [[[Buf(f"KS{s}.K{h}@{c}") for h in (0, 1)] for s in range(nks)] for c in (0, 1)]
+        self.KSS = [[[Buf(f"KS{s}.snap{w}@{c}") for w in range(WARPS)] for s in range(nks)]
+                    for c in (0, 1)]
+        self.KD = [[Buf(f"KD{s}@{c}") for s in range(nkd)] for c in (0, 1)]
+        self.V = [[Buf(f"V{s}@{c}") for s in range(nv)] for c in (0, 1)]
+        self.P = [[[Buf(f"P{s}.{w}@{c}") for w in range(WARPS)] for s in range(npb)] for c in (0, 1)]
+        self.S = [[Buf(f"tmS{f}@{c}", P_ids[c]) for f in range(NF)] for c in (0, 1)]
+        self.O = [[Buf(f"tmO{f}@{c}", O_ids[c]) for f in range(NF)] for c in (0, 1)]
+        self.DKV = [[Buf(f"tmDKV{s}@{c}", KV_ids[c]) for s in range(NDK)] for c in (0, 1)]
         self.ssx = [[[None] * WARPS for _ in range(2)] for _ in (0, 1)]
         self.inflight: list[_Ev] = []
-        self.fifo = {"A": [], "B": []}
-        self.issued = {"A": 0, "B": 0}
-        self.completed = {"A": 0, "B": 0}
+        self.fifo = {"A": [], "D": []}
+        self.issued = {"A": 0, "D": 0}
+        self.completed = {"A": 0, "D": 0}
         self.commits: list[_Ev] = []
 
     @staticmethod
-    def compiles(kk, qh, kv, pbufs, sahead):
-        """The compile-time checks on the ring depths (PairCfg in prefill_pair.cuh and the
-        pair kernel's launch in lightning.cu)."""
-        ns = sahead + 1
-        return (kk <= ns and qh <= NDONE and kv <= NDONE and pbufs <= NDONE
-                and (sahead <= kv or pbufs <= kv))
+    def compiles(nq, nks, nkd, nv, npb):
+        """The kernel's static_asserts on the ring depths (PairCfg in prefill_pair.cuh): a
+        ring's slot of block x is tested free on the done barrier of block x, which must not
+        have been lapped when the producer tests it; and group KV's wait for the value tile
+        of a partial last block (one block before its dKV) is exact only if the slot's
+        previous load fed a dKV that group has seen complete."""
+        return nq <= NF and nks <= NF and nv <= NF and nkd <= NDK and npb <= NF and nv >= 2
 
     # ------------------------------------------------------------------ set-up
     def _cta_bars(self, c):
@@ -159,21 +160,20 @@ class PairModel:
 
         def ring(name, n, count):
             return [Barrier(f"{name}[{i}]@{c}", count) for i in range(n)]
-        single_p = "single_p_ready" in self.mut
         return {
-            "full_kk": ring("full_kk", self.NKK, 1),
-            "full_qh": ring("full_qh", self.NQH, 1),
-            "full_kv": ring("full_kv", self.NKV, 1),
-            "tail_kv": Barrier(f"tail_kv@{c}", 1),
+            "full_q": ring("full_q", self.NQ, 1),
+            "full_ks": ring("full_ks", self.NKS, 1),
+            "full_kd": ring("full_kd", self.NKD, 1),
+            "full_v": ring("full_v", self.NV, 1),
+            "tail_v": Barrier(f"tail_v@{c}", 1),
             "tail_zeroed": Barrier(f"tail_zeroed@{c}", G),
-            "s_full": ring("s_full", self.NS, 1),
-            "s_free": ring("s_free", self.NS, G),
-            "kv_done": ring("kv_done", NDONE, 1),
-            "o_done": ring("o_done", NDONE, 1),
-            "o_free": ring("o_free", 2, G),
-            "dkv_free": ring("dkv_free", 2, G),
-            "p_ready": ring("p_ready", 1 if single_p else self.NPB, G),
-            "snap_ready": ring("snap_ready", 2, G),
+            "f1_done": ring("f1_done", NF, 1),
+            "dkv_done": ring("dkv_done", NDK, 1),
+            "o_done": ring("o_done", NF, 1),
+            "f1_free": ring("f1_free", NF, 2 * G),
+            "dkv_free": ring("dkv_free", NDK, G),
+            "p_ready": ring("p_ready", self.NPB, G),
+            "snap_ready": ring("snap_ready", self.NKS, G),
             "drain": Barrier(f"drain@{c}", 2),
             "ss_bar": ring("ss_bar", 2, WARPS),
         }
@@ -215,6 +215,8 @@ class PairModel:
         buf.zeroed.add(w)
 
     def mma(self, issuer, what, reads, writes, zeroed=()):
+        """writes: (buf, tag, acc, new_tag): an accumulating write expects ``tag`` in the
+        buffer and leaves ``new_tag`` (the next stage of the same accumulator)."""
         for buf, tag in reads:
             if buf.tag != tag or buf.writing:
                 state = " (still being written)" if buf.writing else ""
@@ -224,20 +226,21 @@ class PairModel:
             if buf.zeroed != set(range(WARPS)):
                 raise ProtocolError(f"{issuer}: {what} reads {buf.name} before the rows past the "
                                     f"sequence end were zeroed")
-        for buf, tag, acc in writes:
+        for buf, tag, acc, new_tag in writes:
             if acc:
                 if buf.tag != tag:
                     raise ProtocolError(f"{issuer}: {what} accumulates onto {buf.name} holding "
                                         f"{buf.tag}, wants {tag}")
+                buf.tag = new_tag
             else:
                 if buf.consumers:
                     raise ProtocolError(f"{issuer}: {what} overwrites {buf.name} ({buf.tag}) before "
                                         f"{sorted(buf.consumers)} loaded it")
-                buf.tag, buf.consumers = tag, set(buf.consumer_ids)
+                buf.tag, buf.consumers = new_tag, set(buf.consumer_ids)
             buf.writing += 1
         for buf, _ in reads:
             buf.reading += 1
-        self.fifo[issuer].append((reads, writes))
+        self.fifo[issuer].append((reads, [(b, t, a) for b, t, a, _ in writes]))
         self.issued[issuer] += 1
 
     def commit(self, issuer, targets):
@@ -252,17 +255,20 @@ class PairModel:
             raise ProtocolError(f"{who}: loads {buf.name} ({tag}) twice")
         buf.consumers.discard(wid)
 
+    def _both(self, name, i, phase):
+        return [(self.bars[c][name][i], phase) for c in (0, 1)]
+
     # ------------------------------------------------------------------ agents
     def producer(self, c):
         who = f"producer{c}"
         B0, Bc = self.bars[0], self.bars[c]
-        nb, NKK, NQH, NKV, NS = self.nb, self.NKK, self.NQH, self.NKV, self.NS
-        jk = jq = jv = 0
-        # a query slot is released by O_j (o_done); the mutation releases it at S_j instead
-        if "qh_release_on_s_full" in self.mut:
-            qh_ring, qh_n = Bc["s_full"], NS
+        nb, NQ, NKS, NKD, NV = self.nb, self.NQ, self.NKS, self.NKD, self.NV
+        jq = js = jd = jv = 0
+        # value slots are released by P V (o_done); the mutation releases them at dKV
+        if "v_release_on_dkv" in self.mut:
+            v_ring, v_n = Bc["dkv_done"], NDK
         else:
-            qh_ring, qh_n = Bc["o_done"], NDONE
+            v_ring, v_n = Bc["o_done"], NF
 
         def freed(ring, nring, j, depth):
             x = j - depth
@@ -270,190 +276,197 @@ class PairModel:
                 return True
             bar, n = ring[x % nring], x // nring
             self._check_wait(who, bar, n, start=True)
+            if bar.done > n + 1:   # the parity test would read the lapped phase
+                raise ProtocolError(f"{who}: tests phase {n} of {bar.name} after phase {n + 1} "
+                                    f"completed")
             return bar.done >= n + 1
 
         def cond(ring, nring, j, depth):
             x = j - depth
             return [] if x < 0 else [(ring[x % nring], x // nring)]
 
-        while jk < nb or jq < nb or jv < nb:
+        while jq < nb or js < nb or jd < nb or jv < nb:
             progressed = False
-            if jk < nb and freed(Bc["s_full"], NS, jk, NKK):
-                slot, ph, bar = jk % NKK, jk // NKK, B0["full_kk"][jk % NKK]
+            if jd < nb and freed(Bc["dkv_done"], NDK, jd, NKD):
+                slot, ph, bar = jd % NKD, jd // NKD, B0["full_kd"][jd % NKD]
                 if c == 0:
-                    self.arrive(who, 0, bar, ph, expect_tx=2 * KK_BYTES)
-                for h in (0, 1):
-                    self.tma(who, self.KK[c][slot][h], ("k", jk), bar, ph, HBOX)
-                jk += 1
+                    self.arrive(who, 0, bar, ph, expect_tx=2 * FBOX)
+                self.tma(who, self.KD[c][slot], ("kd", jd), bar, ph, FBOX)
+                jd += 1
                 progressed = True
-            if jq < nb and freed(qh_ring, qh_n, jq, NQH):
-                slot, ph, bar = jq % NQH, jq // NQH, B0["full_qh"][jq % NQH]
-                if c == 0:
-                    self.arrive(who, 0, bar, ph, expect_tx=2 * QH_BYTES)
-                for h in (0, 1):
-                    self.tma(who, self.QH[c][slot][h], ("q", jq), bar, ph, HBOX)
-                jq += 1
-                progressed = True
-            if jv < nb and freed(Bc["kv_done"], NDONE, jv, NKV) and freed(Bc["o_done"], NDONE, jv, NKV):
-                slot, ph = jv % NKV, jv // NKV
+            if jv < nb and freed(v_ring, v_n, jv, NV):
+                slot, ph = jv % NV, jv // NV
                 last_partial = self.tail and jv == nb - 1
                 if c == 0:
-                    bar = B0["full_kv"][slot]
-                    self.arrive(who, 0, bar, ph, expect_tx=(1 if last_partial else 2) * KV_BYTES)
+                    bar = B0["full_v"][slot]
+                    self.arrive(who, 0, bar, ph, expect_tx=(1 if last_partial else 2) * FBOX)
                 elif last_partial:
-                    bar, ph = Bc["tail_kv"], 0
-                    bar.arrive(0, who, KV_BYTES)
+                    bar, ph = Bc["tail_v"], 0
+                    bar.arrive(0, who, FBOX)
                 else:
-                    bar = B0["full_kv"][slot]
-                self.tma(who, self.KV[c][slot]["K"], ("kv", jv), bar, ph, FBOX)
-                self.tma(who, self.KV[c][slot]["V"], ("kv", jv), bar, ph, FBOX)
+                    bar = B0["full_v"][slot]
+                self.tma(who, self.V[c][slot], ("v", jv), bar, ph, FBOX)
                 jv += 1
+                progressed = True
+            if js < nb and freed(Bc["f1_done"], NF, js, NKS):
+                slot, ph, bar = js % NKS, js // NKS, B0["full_ks"][js % NKS]
+                if c == 0:
+                    self.arrive(who, 0, bar, ph, expect_tx=4 * HBOX)
+                for h in (0, 1):
+                    self.tma(who, self.KSK[c][slot][h], ("k", js), bar, ph, HBOX)
+                js += 1
+                progressed = True
+            if jq < nb and freed(Bc["f1_done"], NF, jq, NQ):
+                slot, ph, bar = jq % NQ, jq // NQ, B0["full_q"][jq % NQ]
+                if c == 0:
+                    self.arrive(who, 0, bar, ph, expect_tx=4 * HBOX)
+                for h in (0, 1):
+                    self.tma(who, self.Q[c][slot][h], ("q", jq), bar, ph, HBOX)
+                jq += 1
                 progressed = True
             if progressed:
                 yield STEP
             else:
                 conds = []
-                if jk < nb:
-                    conds.append(cond(Bc["s_full"], NS, jk, NKK))
-                if jq < nb:
-                    conds.append(cond(qh_ring, qh_n, jq, NQH))
+                if jd < nb:
+                    conds.append(cond(Bc["dkv_done"], NDK, jd, NKD))
                 if jv < nb:
-                    conds.append(cond(Bc["kv_done"], NDONE, jv, NKV) + cond(Bc["o_done"], NDONE, jv, NKV))
+                    conds.append(cond(v_ring, v_n, jv, NV))
+                if js < nb:
+                    conds.append(cond(Bc["f1_done"], NF, js, NKS))
+                if jq < nb:
+                    conds.append(cond(Bc["f1_done"], NF, jq, NQ))
                 yield ("poll", conds)
         # drain: the last loads of each ring have landed before the CTA exits
         if c == 0:
-            for j in range(max(0, jk - NKK), jk):
-                yield ("wait", B0["full_kk"][j % NKK], j // NKK)
-            for j in range(max(0, jq - NQH), jq):
-                yield ("wait", B0["full_qh"][j % NQH], j // NQH)
-            for j in range(max(0, jv - NKV), jv):
-                yield ("wait", B0["full_kv"][j % NKV], j // NKV)
+            for ring, n, j in (("full_q", NQ, jq), ("full_ks", NKS, js), ("full_kd", NKD, jd),
+                               ("full_v", NV, jv)):
+                for x in range(max(0, j - n), j):
+                    yield ("wait", B0[ring][x % n], x // n)
         elif self.tail and jv == nb:
-            yield ("wait", Bc["tail_kv"], 0)
+            yield ("wait", Bc["tail_v"], 0)
 
-    def _kk(self, j):
-        return [(self.KK[c][j % self.NKK][h], ("k", j)) for c in (0, 1) for h in (0, 1)]
-
-    def _qh(self, j):
-        return [(self.QH[c][j % self.NQH][h], ("q", j)) for c in (0, 1) for h in (0, 1)]
+    def issuer_d(self):
+        B0 = self.bars[0]
+        nb = self.nb
+        for j in range(nb):
+            last_tail = self.tail and j == nb - 1
+            yield ("wait", B0["full_kd"][j % self.NKD], j // self.NKD)
+            yield ("wait", B0["full_v"][j % self.NV], j // self.NV)
+            if j >= NDK and "no_dkv_free_wait" not in self.mut:
+                yield ("wait", B0["dkv_free"][j % NDK], (j - NDK) // NDK)
+            if last_tail and "no_tail_zeroed_wait" not in self.mut:
+                yield ("wait", B0["tail_zeroed"], 0)
+            reads = [(self.KD[c][j % self.NKD], ("kd", j)) for c in (0, 1)]
+            reads += [(self.V[c][j % self.NV], ("v", j)) for c in (0, 1)]
+            zeroed = [self.V[c][j % self.NV] for c in (0, 1)] if last_tail else []
+            self.mma("D", f"dKV_{j}", reads,
+                     [(self.DKV[c][j % NDK], None, False, ("dkv", j)) for c in (0, 1)], zeroed)
+            self.commit("D", self._both("dkv_done", j % NDK, j // NDK))
+            yield STEP
+        self.commit("D", [(B0["drain"], 0)])
+        yield ("wait", B0["drain"], 0)
 
     def issuer_a(self):
         B0 = self.bars[0]
-        nb, NS = self.nb, self.NS
+        nb, NKS = self.nb, self.NKS
 
-        def stage_in(j):   # S_j = Q_j K_j^T
-            yield ("wait", B0["full_kk"][j % self.NKK], j // self.NKK)
-            yield ("wait", B0["full_qh"][j % self.NQH], j // self.NQH)
-            if j >= NS:
-                yield ("wait", B0["s_free"][j % NS], (j - NS) // NS)
-            self.mma("A", f"S_{j}", self._kk(j) + self._qh(j),
-                     [(self.S[c][j % NS], ("S", j), False) for c in (0, 1)])
-            self.commit("A", [(self.bars[c]["s_full"][j % NS], j // NS) for c in (0, 1)])
+        def f1(j):   # [S_j | O_j] = Q_j [K_j ; snap_j]^T
+            yield ("wait", B0["full_q"][j % self.NQ], j // self.NQ)
+            yield ("wait", B0["full_ks"][j % NKS], j // NKS)
+            yield ("wait", B0["snap_ready"][j % NKS], j // NKS)
+            if j >= NF and "no_f1_free_wait" not in self.mut:
+                yield ("wait", B0["f1_free"][j % NF], (j - NF) // NF)
+            reads = [(self.Q[c][j % self.NQ][h], ("q", j)) for c in (0, 1) for h in (0, 1)]
+            reads += [(self.KSK[c][j % NKS][h], ("k", j)) for c in (0, 1) for h in (0, 1)]
+            reads += [(self.KSS[c][j % NKS][w], ("snap", j)) for c in (0, 1) for w in range(WARPS)]
+            writes = [(self.S[c][j % NF], None, False, ("S", j)) for c in (0, 1)]
+            writes += [(self.O[c][j % NF], None, False, ("oi", j)) for c in (0, 1)]
+            self.mma("A", f"F1_{j}", reads, writes)
+            self.commit("A", self._both("f1_done", j % NF, j // NF))
             yield STEP
 
-        for j in range(min(self.SAHEAD, nb)):
-            yield from stage_in(j)
+        def pv(j):   # O_j += P_j V_j
+            yield ("wait", B0["p_ready"][j % self.NPB], j // self.NPB)
+            yield ("wait", B0["full_v"][j % self.NV], j // self.NV)
+            reads = [(self.P[c][j % self.NPB][w], ("p", j)) for c in (0, 1) for w in range(WARPS)]
+            reads += [(self.V[c][j % self.NV], ("v", j)) for c in (0, 1)]
+            self.mma("A", f"PV_{j}", reads, [(self.O[c][j % NF], ("oi", j), True, ("o", j)) for c in (0, 1)])
+            self.commit("A", self._both("o_done", j % NF, j // NF))
+            yield STEP
+
+        if nb > 0:
+            yield from f1(0)
         for b in range(nb):
-            slot = b % self.NKV
-            zero_tail = self.tail and b == nb - 1
-            if zero_tail and "no_tail_zeroed_wait" not in self.mut:
-                yield ("wait", B0["tail_zeroed"], 0)
-            yield ("wait", B0["full_kv"][slot], b // self.NKV)
-            if b >= 2 and "no_dkv_free_wait" not in self.mut:
-                yield ("wait", B0["dkv_free"][b & 1], (b - 2) >> 1)
-            reads = [(self.KV[c][slot][p], ("kv", b)) for c in (0, 1) for p in ("K", "V")]
-            zeroed = [self.KV[c][slot]["V"] for c in (0, 1)] if zero_tail else []
-            self.mma("A", f"dKV_{b}", reads, [(self.DKV[c][b & 1], ("dkv", b), False) for c in (0, 1)],
-                     zeroed)
-            self.commit("A", [(self.bars[c]["kv_done"][b % NDONE], b // NDONE) for c in (0, 1)])
-            yield STEP
-            if b + self.SAHEAD < nb:
-                yield from stage_in(b + self.SAHEAD)
+            if b + 1 < nb:
+                yield from f1(b + 1)
+            yield from pv(b)
         self.commit("A", [(B0["drain"], 0)])
-        yield ("wait", B0["drain"], 0)
-
-    def _snap(self, u):
-        return [(self.SNAP[c][u % self.NSNAP][w], ("snap", u)) for c in (0, 1) for w in range(WARPS)]
-
-    def _snap_ready(self, u):
-        if self.NSNAP == 1:
-            return self.bars[0]["snap_ready"][0], u - self.u0
-        return self.bars[0]["snap_ready"][u & 1], (u - self.u0) >> 1
-
-    def _p_ready(self, b):
-        if "single_p_ready" in self.mut:
-            return self.bars[0]["p_ready"][0], b
-        return self.bars[0]["p_ready"][b % self.NPB], b // self.NPB
-
-    def issuer_b(self):
-        B0 = self.bars[0]
-        for b in range(self.nb):
-            if b >= 2:
-                yield ("wait", B0["o_free"][b & 1], (b - 2) >> 1)
-            if "no_qh_wait_b" not in self.mut:
-                yield ("wait", B0["full_qh"][b % self.NQH], b // self.NQH)
-            if b >= self.u0:
-                yield ("wait", *self._snap_ready(b))
-                self.mma("B", f"Qsnap_{b}", self._qh(b) + self._snap(b),
-                         [(self.O[c][b & 1], ("o", b), False) for c in (0, 1)])
-                yield STEP
-            yield ("wait", *self._p_ready(b))
-            yield ("wait", B0["full_kv"][b % self.NKV], b // self.NKV)
-            reads = [(self.P[c][b % self.NPB][w], ("p", b)) for c in (0, 1) for w in range(WARPS)]
-            reads += [(self.KV[c][b % self.NKV]["V"], ("kv", b)) for c in (0, 1)]
-            self.mma("B", f"PV_{b}", reads, [(self.O[c][b & 1], ("o", b), b >= self.u0) for c in (0, 1)])
-            self.commit("B", [(self.bars[c]["o_done"][b % NDONE], b // NDONE) for c in (0, 1)])
-            yield STEP
-        self.commit("B", [(B0["drain"], 0)])
         yield ("wait", B0["drain"], 0)
 
     def group_p(self, c, w):
         who = f"P{c}.{w}"
         B0, Bc = self.bars[0], self.bars[c]
-        NS = self.NS
-        for b in range(self.nb):
-            yield ("wait", Bc["s_full"][b % NS], b // NS)
-            self.tmem_ld(who, ("P", c, w), self.S[c][b % NS], ("S", b))
-            self.arrive(who, c, B0["s_free"][b % NS], b // NS)
+        for j in range(self.nb):
+            yield ("wait", Bc["f1_done"][j % NF], j // NF)
+            self.tmem_ld(who, ("P", c, w), self.S[c][j % NF], ("S", j))
+            self.arrive(who, c, B0["f1_free"][j % NF], j // NF)
             yield STEP
-            pb = b - self.NPB
+            pb = j - self.NPB
             if pb >= 0 and "no_o_done_wait_p" not in self.mut:
-                yield ("wait", Bc["o_done"][pb % NDONE], pb // NDONE)
-            self.store(who, self.P[c][b % self.NPB][w], ("p", b))
+                yield ("wait", Bc["o_done"][pb % NF], pb // NF)
+            self.store(who, self.P[c][j % self.NPB][w], ("p", j))
+            self.arrive(who, c, B0["p_ready"][j % self.NPB], j // self.NPB)
             yield STEP
-            if self.tail and b == self.nb - 1:
-                if c == 0:
-                    yield ("wait", B0["full_kv"][b % self.NKV], b // self.NKV)
-                else:
-                    yield ("wait", Bc["tail_kv"], 0)
-                self.zero_tail(who, w, self.KV[c][b % self.NKV]["V"], ("kv", b))
-                self.arrive(who, c, B0["tail_zeroed"], 0)
+
+    def group_kv(self, c, w):
+        who = f"KV{c}.{w}"
+        B0, Bc = self.bars[0], self.bars[c]
+        nb, NKS = self.nb, self.NKS
+
+        def write_snap(u):
+            self.store(who, self.KSS[c][u % NKS][w], ("snap", u))
+            self.arrive(who, c, B0["snap_ready"][u % NKS], u // NKS)
+
+        def zero_tail():
+            b = nb - 1
+            if c == 0:
+                yield ("wait", B0["full_v"][b % self.NV], b // self.NV)
+            else:
+                yield ("wait", Bc["tail_v"], 0)
+            self.zero_tail(who, w, self.V[c][b % self.NV], ("v", b))
+            self.arrive(who, c, B0["tail_zeroed"], 0)
+            yield STEP
+
+        if nb > 0:
+            write_snap(0)
+            yield STEP
+            if self.tail and nb == 1:
+                yield from zero_tail()
+        for b in range(nb):
+            if self.tail and nb >= 2 and b == nb - 2:
+                yield from zero_tail()
+            yield ("wait", Bc["dkv_done"][b % NDK], b // NDK)
+            self.tmem_ld(who, ("KV", c, w), self.DKV[c][b % NDK], ("dkv", b))
+            self.arrive(who, c, B0["dkv_free"][b % NDK], b // NDK)
+            yield STEP
+            if b + 1 < nb:
+                x = b + 1 - NKS
+                if x >= 0 and "no_snap_slot_wait" not in self.mut:
+                    yield ("wait", Bc["f1_done"][x % NF], x // NF)
+                write_snap(b + 1)
                 yield STEP
-            self.arrive(who, c, *self._p_ready(b))
-            yield STEP
 
     def group_o(self, c, w):
         who = f"O{c}.{w}"
         B0, Bc = self.bars[0], self.bars[c]
-
-        def write_snap(u):
-            self.store(who, self.SNAP[c][u % self.NSNAP][w], ("snap", u))
-            self.arrive(who, c, *self._snap_ready(u))
-
-        if self.init:
-            write_snap(0)
-            yield STEP
         for b in range(self.nb):
-            yield ("wait", Bc["kv_done"][b % NDONE], b // NDONE)
-            self.tmem_ld(who, ("O", c, w), self.DKV[c][b & 1], ("dkv", b))
-            self.arrive(who, c, B0["dkv_free"][b & 1], b >> 1)
-            yield STEP
-            if b + 1 < self.nb:
-                write_snap(b + 1)
-                yield STEP
-            yield ("wait", Bc["o_done"][b % NDONE], b // NDONE)
-            self.tmem_ld(who, ("O", c, w), self.O[c][b & 1], ("o", b))
-            self.arrive(who, c, B0["o_free"][b & 1], b >> 1)
+            if "o_after_f1" in self.mut:      # waits for F1_b instead of P_b V_b
+                yield ("wait", Bc["f1_done"][b % NF], b // NF)
+            else:
+                yield ("wait", Bc["o_done"][b % NF], b // NF)
+            self.tmem_ld(who, ("O", c, w), self.O[c][b % NF], ("o", b))
+            self.arrive(who, c, B0["f1_free"][b % NF], b // NF)
             yield STEP
             if self.rms:   # exchange of the row's partial sum of squares with warp w ^ 2
                 prev = self.ssx[c][b & 1][w]
@@ -473,17 +486,18 @@ class PairModel:
     def agents(self):
         """name -> generator, one per role of the kernel."""
         agents = {"producer0": self.producer(0), "producer1": self.producer(1),
-                  "A": self.issuer_a(), "B": self.issuer_b()}
+                  "A": self.issuer_a(), "D": self.issuer_d()}
         for c in (0, 1):
             for w in range(WARPS):
                 agents[f"P{c}.{w}"] = self.group_p(c, w)
+                agents[f"KV{c}.{w}"] = self.group_kv(c, w)
                 agents[f"O{c}.{w}"] = self.group_o(c, w)
         return agents
 
     # ------------------------------------------------------------------ scheduler
     def _events(self):
         evs = list(self.inflight)
-        for who in ("A", "B"):
+        for who in ("A", "D"):
             if self.fifo[who]:
                 evs.append(_Ev("mma", who))
         evs += [e for e in self.commits if self.completed[e.args[0]] >= e.args[1]]
@@ -569,5 +583,5 @@ class PairModel:
                             self._check_wait(n, bar, k, start=False)
         else:
             raise ProtocolError("no end after max_steps")
-        if self.inflight or self.fifo["A"] or self.fifo["B"] or self.commits:
+        if self.inflight or self.fifo["A"] or self.fifo["D"] or self.commits:
             raise ProtocolError("work still in flight after every agent finished")

@@ -1,20 +1,21 @@
 """The paired prefill kernel's barrier protocol, checked on the CPU by its executable model
-(``pair_protocol.py``): random schedules of the producer, the two MMA issuers and the
+(``pair_protocol.py``): random schedules of the producers, the two MMA issuers and the
 epilogue warps of both CTAs, with TMA landings, MMA completions, commit arrivals and
 remote arrivals in random order.
 
 Three things are checked:
   * the kernel's protocol is clean (no parity-alias, data or ordering violation, no
     deadlock) for every block count shape (empty, one block, partial last block, initial
-    state, RMSNorm) and for every ring depth the kernel's static_asserts accept;
-  * the ring depths those asserts reject do fail in the model, where they can;
-  * each planted protocol mistake (one wait or barrier taken out or merged) is caught.
+    state, RMSNorm) and for every ring depth the kernel's static_assert accepts;
+  * ring depths that assert rejects do fail in the model;
+  * each planted protocol mistake (one wait taken out, a slot released by the wrong
+    product, the output loaded after the wrong product) is caught.
 """
 import itertools
 
 import pytest
 
-from pair_protocol import PairModel, ProtocolError
+from pair_protocol import NDK, NF, PairModel, ProtocolError
 
 SEEDS = 8
 
@@ -28,23 +29,21 @@ def test_default_rings(nb, tail, init, rms):
         PairModel(nb, tail=tail, init=init, rms=rms).run(seed)
 
 
-def _depths():
-    for sahead in (1, 2):
-        for kk, qh, kv, pb in itertools.product(range(1, sahead + 2), range(1, 5), range(1, 5),
-                                                range(1, 5)):
-            yield kk, qh, kv, pb, sahead
+def _depths(hi=4):
+    return itertools.product(range(1, hi + 1), range(1, hi + 1), range(1, hi), range(1, hi + 1),
+                             range(1, hi + 1))
 
 
 def test_every_accepted_ring_depth():
     accepted = [d for d in _depths() if PairModel.compiles(*d)]
-    assert (2, 4, 2, 1, 1) in accepted            # the kernel's default depths
-    for i, (kk, qh, kv, pb, sahead) in enumerate(accepted):
-        for nb, seed in ((3, i), (6, i + 1)):
-            PairModel(nb, tail=True, init=bool(seed & 1), rms=bool(seed & 2), kk=kk, qh=qh, kv=kv,
-                      pbufs=pb, sahead=sahead).run(seed)
+    assert (2, 2, 2, 3, 2) in accepted            # the kernel's depths
+    for i, (nq, nks, nkd, nv, npb) in enumerate(accepted):
+        for nb, seed in ((3, i), (7, i + 1)):
+            PairModel(nb, tail=bool(seed & 1), init=bool(seed & 2), rms=bool(seed & 4), nq=nq,
+                      nks=nks, nkd=nkd, nv=nv, npb=npb).run(seed)
 
 
-def _first_violation(seeds=200, **kw):
+def _first_violation(seeds=300, **kw):
     for seed in range(seeds):
         try:
             PairModel(**kw).run(seed)
@@ -53,43 +52,44 @@ def _first_violation(seeds=200, **kw):
     return None
 
 
-def test_rejected_ring_depths_do_fail():
-    """Look-ahead 2 with one K/V slot and two or more P buffers: CTA 0's group P may start its
-    wait on the partial last block's load while the slot's previous phase is still open.
-    The check is conservative for a single query slot: then S_b cannot start before
-    O_{b-1} has completed, which implies that load, and the model finds nothing."""
-    rejected = [d for d in _depths() if not PairModel.compiles(*d)]
-    assert rejected and all(d[4] == 2 and d[2] == 1 and d[3] >= 2 for d in rejected)
-    for kk, qh, kv, pb, sahead in rejected:
-        with pytest.raises(ValueError):
-            PairModel(3, kk=kk, qh=qh, kv=kv, pbufs=pb, sahead=sahead)
-        msg = _first_violation(nb=3, tail=True, kk=kk, qh=qh, kv=kv, pbufs=pb, sahead=sahead,
-                               static_checks=False)
-        if qh == 1:
-            assert msg is None, (kk, qh, kv, pb, sahead, msg)
-        else:
-            assert msg is not None and "full_kv" in msg, (kk, qh, kv, pb, sahead)
+@pytest.mark.parametrize("depths,barrier", [
+    (dict(nkd=NDK + 1), "dkv_done"),      # key-dim slots tested on a 2-deep dkv_done ring
+    (dict(nq=NF + 1), "f1_done"),         # query slots tested on the f1_done ring
+    (dict(nv=1), "full_v"),               # group KV's tail wait meets an open previous phase
+])
+def test_rejected_ring_depths_do_fail(depths, barrier):
+    """A ring deeper than the done-barrier ring its slots are released on: the producer's
+    test of a slot can meet a barrier already lapped by the block one ring further on.  And
+    a one-slot value ring: group KV's wait for the partial last block's value tile starts
+    while the slot's previous phase is still open.  (For a 4-deep value ring on the 3-deep
+    o_done ring the bound is conservative: lapping there needs P V of the block before to
+    complete while the producer has not yet tested the slot, and the model finds no such
+    schedule.)"""
+    with pytest.raises(ValueError):
+        PairModel(6, **depths)
+    msg = _first_violation(nb=8, tail=True, static_checks=False, **depths)
+    assert msg is not None and (barrier in msg or "deadlock" in msg), (depths, msg)
 
 
 # mutation -> (shape, words of which the first violation must name one: the mistake's symptoms)
 MUTANTS = {
-    # issuer B issues Q_b snap_b without waiting for the query tile to land
-    "no_qh_wait_b": (dict(nb=4, init=True), ("QH",)),
-    # issuer A overwrites a dKV accumulator before group O loaded it
-    "no_dkv_free_wait": (dict(nb=5), ("tmDKV",)),
-    # group P stores P_b before P_{b-1} V has completed
-    "no_o_done_wait_p": (dict(nb=4), ("p_ready", "P0.", "P1.")),
-    # two P buffers behind one p_ready barrier (phases alias)
-    "single_p_ready": (dict(nb=5, pbufs=2), ("p_ready",)),
-    # issuer A reads the partial last block before group P zeroed its value rows (and, in
-    # CTA 1, before its tiles landed: only the zeroing implies that)
-    "no_tail_zeroed_wait": (dict(nb=3, tail=True), ("zeroed", "KV")),
-    # one snapshot buffer: snapshot b+1 overwrites snapshot b under Q_b snap_b, and the
-    # buffer's one barrier aliases phases
-    "one_snapshot": (dict(nb=5), ("SNAP", "snap_ready")),
-    # query slots released when S_j completes, though Q_j snap_j still reads them (and the
-    # 4-deep query ring then laps the 2-deep s_full ring)
-    "qh_release_on_s_full": (dict(nb=5), ("full_qh", "QH", "s_full")),
+    # the dKV issuer overwrites a dKV accumulator before group KV loaded it
+    "no_dkv_free_wait": (dict(nb=6), ("tmDKV",)),
+    # the F1 issuer overwrites an [S | O] region before groups P and O loaded it
+    "no_f1_free_wait": (dict(nb=7), ("tmS", "tmO", "f1_free")),
+    # group P stores P_j before P_{j-1} V has completed (one P buffer: with two, F1_j's
+    # completion, which group P waits for, already implies P_{j-2} V's, as one thread issues
+    # both in that order)
+    "no_o_done_wait_p": (dict(nb=5, npb=1), ("P0.", "P1.", "p_ready")),
+    # dKV reads the partial last block before group KV zeroed its value rows (and, in
+    # CTA 1, before its tile landed: only the zeroing implies that)
+    "no_tail_zeroed_wait": (dict(nb=3, tail=True), ("zeroed", "V")),
+    # group KV writes the next snapshot into a key-row slot that F1 still reads
+    "no_snap_slot_wait": (dict(nb=6), ("KS", "snap")),
+    # value slots released when dKV completes, though P V still reads them
+    "v_release_on_dkv": (dict(nb=6), ("V", "full_v", "dkv_done")),
+    # group O loads O_b once F1_b completes, before P_b V_b has added to it
+    "o_after_f1": (dict(nb=4), ("tmO",)),
 }
 
 
