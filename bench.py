@@ -46,6 +46,7 @@ WORKLOADS = {
     # name: (B, N, H, D, beta)
     "prefill_n131k": (1, 131072, 64, 128, 128),
     "prefill_n16k": (1, 16384, 64, 128, 128),
+    "prefill_n16k_b64": (1, 16384, 64, 128, 64),
 }
 DECODE = dict(B=256, H=64, D=128, N=4096, steps=64, chunk=32)
 KERNEL_SOURCES = [os.path.join(ROOT, "long_context_04_b200", "csrc", f)
