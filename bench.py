@@ -14,9 +14,12 @@ prefill kernel, the end-to-end number through the C ABI with host buffers, a
 sweep of the sequence length at a fixed token count, and the fp64 oracle timed on
 the host cores as a CPU baseline.
 
-Multi-GPU (torchrun): every rank runs its own copy of the workload on its own
-GPU (independent problems, no data-path collective: weak scaling); the timed
-region is bracketed by barriers and the slowest rank's time is reported.
+Multi-GPU (torchrun): the heads are independent units, so N ranks run a layer of
+64 N heads, 64 heads per rank, with no data-path collective (weak scaling); the
+timed region is bracketed by barriers and the slowest rank's time is reported.
+The ``lasp`` key adds LASP+ sequence parallelism (strong scaling): one sequence
+of N=131072 tokens split into N contiguous chunks, with one all-gather of the
+chunk states between the chunk-state and the prefill kernels.
 
 ``--impl reference`` times the fp64 CPU oracle on the same metric and unit,
 each step a bounded sample of the workload (rank 0 only).
@@ -382,10 +385,13 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic: Q, K, V iid N(0,1)/sqrt(D), seeded per rank",
-        "config": {"workload": workload_name(args.workload), "global_batch": B * world,
+        "data": "synthetic: Q, K, V iid N(0,1)/sqrt(D), seeded per head shard (rank)",
+        "config": {"workload": workload_name(args.workload), "global_batch": B,
                    "seq_len": N, "heads": H, "head_dim": D, "beta": beta,
-                   "parallelism": f"replicas x{world} (independent problems, no collective)",
+                   "heads_total": H * world,
+                   "parallelism": (f"heads sharded x{world}: a layer of {H * world} heads, "
+                                   f"{H} per rank, no collective" if world > 1 else
+                                   "one GPU, no collective"),
                    "l2": "inputs (8.6 GB) larger than the 126 MB L2; no flush"},
         "prefill": prefill_view, "roofline": roofline, "gpu_launches": args.steps,
         "clocks": clk.summary(),
@@ -402,6 +408,13 @@ def run_ours(args):
                 line["decode"]["cpu_baseline"] = {"error": repr(e)}
         del dctx
         line["lasp_chunk_state"] = bench_chunk_state(api, torch, stream, k, v, peak_bw, world)
+        if world > 1:   # every rank must reach the same collectives: no local recovery
+            line["lasp"] = lasp_leg(api, torch, stream, q, k, v, o, rank, world, peak_bw, dev)
+        else:
+            try:
+                line["lasp"] = lasp_leg(api, torch, stream, q, k, v, o, rank, world, peak_bw, dev)
+            except Exception as e:  # an extra that fails must not cost the main line
+                line["lasp"] = {"error": repr(e)}
         if world == 1:  # rank-local extra: no collective, so a failure cannot strand other ranks
             try:
                 line["length_sweep"] = bench_length_sweep(api, torch, stream, q, k, v, o, beta, peak_bw)
@@ -557,32 +570,41 @@ def bench_length_sweep(api, torch, stream, q, k, v, o, beta, peak_bw, reps=20, w
 
 
 def bench_prefill_options(api, torch, stream, q, k, v, o, peak_bw, reps=10, warm=3):
-    """The main workload through the other options of la_prefill, each timed alone: the fused
-    output RMSNorm, beta = 64 (the unpaired tcgen05 kernel) and a start from an initial
-    state (read only; the inter-block term of block 0 is then computed too)."""
+    """The main workload through the other options of la_prefill: the fused output RMSNorm,
+    beta = 64 (the unpaired tcgen05 kernel) and a start from an initial state (read only;
+    the inter-block term of block 0 is then computed too).  The options and the plain call
+    take turns launch by launch, so that each option meets the same clocks and power state
+    as the plain launches it is compared with (``vs_plain`` = median over median)."""
     H, D = q.shape[-2], q.shape[-1]
     T = q.numel() // (H * D)
     S = q.shape[0] if q.dim() == 4 else 1
     X = torch.zeros((S, H, D, D), dtype=torch.float32, device=q.device)
-    cases = {"rmsnorm": dict(beta=128, rmsnorm=True),
+    cases = {"plain": dict(beta=128),
+             "rmsnorm": dict(beta=128, rmsnorm=True),
              "beta64": dict(beta=64),
              "initial_state": dict(beta=128, initial_state=X)}
+    for _ in range(warm):
+        for kw in cases.values():
+            api.prefill(q, k, v, out=o, stream=stream, **kw)
+    ev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(reps)] for name in cases}
+    torch.cuda.synchronize()
+    for i in range(reps):
+        for name, kw in cases.items():
+            ev[name][i][0].record(stream)
+            api.prefill(q, k, v, out=o, stream=stream, **kw)
+            ev[name][i][1].record(stream)
+    stream.synchronize()
+    med = {name: statistics.median(a.elapsed_time(b) for a, b in ev[name]) for name in cases}
     res = {}
-    for name, kw in cases.items():
-        for _ in range(warm):
-            api.prefill(q, k, v, out=o, stream=stream, **kw)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(reps):
-            api.prefill(q, k, v, out=o, stream=stream, **kw)
-        e1.record(stream)
-        stream.synchronize()
-        ms = e0.elapsed_time(e1) / reps
+    for name in cases:
+        ms = med[name]
         res[name] = {"ms_per_launch": ms, "tokens_per_s": T / (ms / 1e3),
                      "hbm_frac": prefill_bytes(T, H, D) / (ms / 1e3) / 1e9 / peak_bw,
-                     "status": api.status_string(api.device_status(stream))}
+                     "vs_plain": ms / med["plain"]}
+    res["status"] = api.status_string(api.device_status(stream))
     res["launches_per_option"] = reps
+    res["order"] = "interleaved: " + ", ".join(cases) + " in turn, medians"
     return res
 
 
@@ -790,6 +812,106 @@ def bench_chunk_state(api, torch, stream, k, v, peak_bw, world, reps=5):
     return {"kernel": "la::chunk_state_tc_kernel (the local state of a chunk in LASP+)",
             "ms_median": ms, "bytes": nbytes, "gbs": gbs, "pct_hbm": 100.0 * gbs / peak_bw,
             "launches": reps, "status": api.status_string(api.device_status(stream))}
+
+
+def dist_gather(values, world: int, device=None):
+    """Every rank's list of floats (same length on every rank), in rank order."""
+    if world == 1:
+        return [list(values)]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    out = t.new_empty((world * t.numel(),))
+    dist.all_gather_into_tensor(out, t)
+    return out.view(world, -1).tolist()
+
+
+LASP_PARTS = ("chunk_state", "all_gather", "state_prefix", "prefill", "step")
+
+
+def lasp_leg(api, torch, stream, q, k, v, o, rank, world, peak_bw, dev):
+    """bench_lasp on the first N / world rows of this rank's inputs ([1, N, H, D] views), as
+    chunk r of one sequence.  On one GPU the leg runs in a one-rank NCCL group of its own,
+    so that the same all-gather on the kernels' stream is exercised."""
+    import datetime
+
+    import torch.distributed as dist
+
+    from long_context_04_b200 import lasp
+    L = q.shape[1] // world
+    views = [x[:, :L] for x in (q, k, v, o)]
+    own = False
+    if world == 1 and not dist.is_initialized():
+        dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+        own = True
+    try:
+        return bench_lasp(api, lasp, torch, stream, *views, rank, world, peak_bw, device=dev)
+    finally:
+        if own:
+            dist.destroy_process_group()
+
+
+def bench_lasp(api, lasp, torch, stream, q, k, v, o, rank, world, peak_bw, device=None,
+               beta=128, reps=10, warm=3):
+    """LASP+ sequence parallelism over the ranks: one sequence of world * L tokens in
+    contiguous chunks, chunk r (q, k, v, o: [1, L, H, D]) on rank r.  One step, in order on
+    the kernels' stream:
+        la_chunk_state   S_r = K_r^T V_r
+        all-gather       the fp32 chunk states of every rank (NCCL, H D^2 4 bytes per rank)
+        la_state_prefix  X_r = sum of S_r' over r' < r
+        la_prefill       O_r from X_r (LA_READ_STATE)
+    Every rank takes the same collectives in the same order.  Reported: each rank's median
+    time of every part, and the whole sequence's tokens/s over the slowest rank's time."""
+    H, D = q.shape[-2], q.shape[-1]
+    L = q.shape[1]
+    local = api.chunk_state(k, v, stream=stream)          # warm-up and allocation
+    init = local.new_zeros(local.shape)
+
+    def step(marks=None):
+        api.chunk_state(k, v, state_out=local, stream=stream)
+        if marks:
+            marks[1].record(stream)
+        gathered = lasp.all_gather_states(local)
+        if marks:
+            marks[2].record(stream)
+        api.state_prefix(gathered, rank, out=init, stream=stream)
+        if marks:
+            marks[3].record(stream)
+        api.prefill(q, k, v, beta=beta, out=o, initial_state=init, stream=stream)
+        if marks:
+            marks[4].record(stream)
+
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):     # the collective is ordered with the kernels
+        for _ in range(warm):
+            step()
+        dist_barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(reps):
+            marks[i][0].record(stream)
+            step(marks[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    dist_barrier(world)
+    total_ms = dist_max(t0.elapsed_time(t1), world, device)
+    parts = [statistics.median(m[j].elapsed_time(m[j + 1]) for m in marks) for j in range(4)]
+    parts.append(statistics.median(m[0].elapsed_time(m[4]) for m in marks))
+    per_rank = dist_gather(parts, world, device)
+    status = api.status_string(api.device_status(stream))
+    tokens = world * L
+    return {"workload": f"one sequence of N={tokens} tokens, H={H}, D={D}, beta={beta}, bf16, "
+                        f"in {world} contiguous chunks of {L} tokens, chunk r on rank r",
+            "steps": reps, "warmup": warm,
+            "slowest_rank_ms_per_step": total_ms / reps,
+            "tokens_per_s": tokens * reps / (total_ms / 1e3),
+            "per_rank_ms_median": [dict(zip(LASP_PARTS, r)) for r in per_rank],
+            "gathered_bytes_per_rank": world * H * D * D * 4,
+            "prefill_hbm_frac": prefill_bytes(L, H, D) / (parts[3] / 1e3) / 1e9 / peak_bw,
+            "scaling": "strong (the sequence is fixed; each rank takes 1/N of it)",
+            "status": status}
 
 
 def bench_concurrent(api, torch, pstream, dctx, q, k, v, o, beta, world, n_prefill=2):

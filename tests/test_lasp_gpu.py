@@ -97,3 +97,30 @@ def test_lasp_ranks_in_sequence(dtype, D, rmsnorm):
     ref_o, ref_s = oracle.recurrent(q, k, v, cu_full, rmsnorm=rmsnorm)
     assert oracle.max_rel_l2_per_head(o, ref_o, cu_full) <= TOL[dtype]
     assert _state_err(final.cpu().numpy(), ref_s) <= STOL[dtype]
+
+
+def test_lasp_prefill_one_nccl_rank():
+    """lasp.lasp_prefill itself on a one-rank NCCL group, on a side stream: the all-gather
+    runs on the kernels' stream between la_chunk_state and la_state_prefix, and the rows and
+    the final state match the oracle's single pass (three packed sequences, bf16, D = 128)."""
+    import datetime
+
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group is already set up in this process")
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        H, D = 4, 128
+        cu = [0, 1000, 1000, 2333]
+        q, k, v = synth.qkv(cu[-1], H, D, seed=45, dtype=torch.bfloat16, device="cuda")
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        o, st = lasp.lasp_prefill(q, k, v, cu_seqlens=cu, return_state=True, stream=s)
+        s.synchronize()
+        assert api.device_status(s) == api.LA_OK
+    finally:
+        dist.destroy_process_group()
+    ref_o, ref_s = oracle.recurrent(q, k, v, cu)
+    assert oracle.max_rel_l2_per_head(o, ref_o, cu) <= TOL[torch.bfloat16]
+    assert _state_err(st.cpu().numpy(), ref_s) <= STOL[torch.bfloat16]
