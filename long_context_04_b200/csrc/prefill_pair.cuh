@@ -39,7 +39,8 @@
 //   warps 2..5   group P (S -> causal mask -> bf16 P in shared memory)
 //   warps 6..9   group KV (KV^T += dKV^T in registers, bf16 snapshot into the key-row
 //                slot of the next block, final state)
-//   warps 10..13 group O (O -> optional RMSNorm -> bf16, TMA store)
+//   warps 10..13 group O (O -> optional RMSNorm -> bf16, TMA store; frees the value
+//                slot of each block once P V has completed)
 //   warp 14      CTA 0: issuer of dKV
 // Each epilogue group has one warp per TMEM sub-partition (warp w reads lanes
 // 32 (w mod 4) .. + 31).  Every wait is bounded; on a timeout the CTA records
@@ -75,15 +76,18 @@ struct PairCfg {
     //   KS: per dim half 128 rows: own 64 key rows (TMA), then own 64 rows of
     //       the snapshot KV^T (group KV) (B of F1)                           f1_done
     //   KD: 128 key rows x own 64 dims (B of dKV^T)                          dkv_done
-    //   V : 128 value rows x own 64 columns (A of dKV^T, B of P V)           o_done
+    //   V : 128 value rows x own 64 columns (A of dKV^T, B of P V)           v_free
     //   P : own 64 rows of P, both key halves (A of P V)                     o_done
-    // (a value tile is released by P V, which follows its dKV in every schedule)
-    static constexpr int NQ = 2, NKS = 2, NKD = 2, NV = 3, NPB = 2;
+    // (a value tile is released once group O has seen P V complete; P V follows its
+    // dKV in every schedule.  Its own release ring lets the value ring run deeper than
+    // the three F1 regions, so that dKV, which feeds the snapshot chain, rarely waits
+    // for a value tile.  One P buffer: group P stores P_b while F1_{b+1} runs.)
+    static constexpr int NQ = 2, NKS = 2, NKD = 2, NV = 4, NPB = 1;
     static constexpr int NF = 3;                        // F1 TMEM regions (S | O)
     static constexpr int NDK = 2;                       // dKV TMEM buffers
     // A ring's slot of block x is tested free on the done barrier of block x, which
     // must not have been lapped (by block x + ring size) when the producer tests it.
-    static_assert(NQ <= NF && NKS <= NF && NV <= NF && NKD <= NDK && NPB <= NF, "release rings");
+    static_assert(NQ <= NF && NKS <= NF && NKD <= NDK && NPB <= NF, "release rings");
     // Group KV waits for the value tile of a partial last block one block before its dKV:
     // the wait is exact only if the slot's previous load fed a dKV it has seen complete.
     static_assert(NV >= 2, "value ring: group KV's tail wait");
@@ -127,6 +131,8 @@ struct PairMisc {
     uint64_t f1_done[PairCfg::NF];   // F1_j complete (region j % NF)
     uint64_t dkv_done[PairCfg::NDK]; // dKV_j complete (buffer j % NDK)
     uint64_t o_done[PairCfg::NF];    // P_j V_j complete (region j % NF)
+    // each CTA's own: its group O has seen P_j V_j complete, value slot j % NV is free
+    uint64_t v_free[PairCfg::NV];
     // used in CTA 0: epilogue -> issuers (arrivals from both CTAs)
     uint64_t f1_free[PairCfg::NF];   // groups P and O have loaded S_j and O_j
     uint64_t dkv_free[PairCfg::NDK]; // group KV has loaded dKV_j
@@ -134,7 +140,6 @@ struct PairMisc {
     uint64_t snap_ready[PairCfg::NKS];  // snapshot u (the state before block u) in slot u % NKS
     uint64_t drain;
     uint64_t done0;                // phase 0 completed at the start: a wait that always passes
-    uint64_t ss_bar[2];            // group O: RMSNorm partial sums written (per block parity)
     uint32_t tmem_base;
     int abort_flag;
     float ss_x[2][2][64];          // RMSNorm partial sums [block parity][column half][row]
@@ -171,7 +176,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             mbar_init(&m->snap_ready[s], BOTH);
         }
         for (int s = 0; s < C::NKD; ++s) mbar_init(&m->full_kd[s], 1);
-        for (int s = 0; s < C::NV; ++s) mbar_init(&m->full_v[s], 1);
+        for (int s = 0; s < C::NV; ++s) {
+            mbar_init(&m->full_v[s], 1);
+            mbar_init(&m->v_free[s], 1);
+        }
         for (int s = 0; s < C::NF; ++s) {
             mbar_init(&m->f1_done[s], 1);
             mbar_init(&m->o_done[s], 1);
@@ -187,8 +195,6 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         mbar_init(&m->drain, 2);
         mbar_init(&m->done0, 1);
         mbar_arrive(&m->done0);
-        mbar_init(&m->ss_bar[0], C::GROUP);
-        mbar_init(&m->ss_bar[1], C::GROUP);
         m->abort_flag = 0;
         fence_mbarrier_init_cluster();
         tma_prefetch_desc(&p.tmap_q64);
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
                     ++jd;
                     progressed = true;
                 }
-                if (jv < nb && freed(m->o_done, C::NF, jv, C::NV)) {
+                if (jv < nb && freed(m->v_free, C::NV, jv, C::NV)) {
                     uint64_t *fb = &m->full_v[jv % C::NV];
                     const uint32_t dst = v_addr(jv);
                     const int row = seq_start + jv * C::BETA;
@@ -610,40 +616,55 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         bool ok = true;
         for (int b = 0; b < nb; ++b) {
             // o_done[b % NF] phase b / NF; the next phase (P V of block b + NF) needs
-            // F1_{b+NF}, which needs f1_free from the load below
-            if (!wwait(&m->o_done[b % C::NF], (uint32_t)((b / C::NF) & 1))) {
+            // F1_{b+NF}, which needs f1_free from the load below.  After a failed wait
+            // the warp still meets the group's named barrier in every block (so no warp
+            // of the group waits there for ever) but skips every other step.
+            if (ok && !wwait(&m->o_done[b % C::NF], (uint32_t)((b / C::NF) & 1))) {
                 ok = false;
-                break;
+                fail();
             }
-            tc_fence_after();
             uint32_t a[32], c[32];
-            const uint32_t tO = tmem + C::TM_F1 + 128 * (b % C::NF) + 64 + lane_base;
-            tmem_ld32(tO, a);
-            tmem_ld32(tO + 32, c);
-            tmem_ld_wait();
-            tc_fence_before();
-            arrive_leader_free(&m->f1_free[b % C::NF]);
+            if (ok) {
+                // v_free[b % NV] phase b / NV; its next phase needs P V of block b + NV,
+                // which reads the value tile the producer loads after this arrival
+                if (q == 0 && lane == 0) mbar_arrive(&m->v_free[b % C::NV]);
+                tc_fence_after();
+                const uint32_t tO = tmem + C::TM_F1 + 128 * (b % C::NF) + 64 + lane_base;
+                tmem_ld32(tO, a);
+                tmem_ld32(tO + 32, c);
+                tmem_ld_wait();
+                tc_fence_before();
+                arrive_leader_free(&m->f1_free[b % C::NF]);
+            }
             float scale = 1.0f;
             if (p.rmsnorm) {
                 float ss = 0.f;
+                if (ok) {
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f};   // four chains: 16 dependent FMAs each
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const float x = __uint_as_float(a[t]), y = __uint_as_float(c[t]);
-                    ss = fmaf(x, x, ss);
-                    ss = fmaf(y, y, ss);
+                    for (int t = 0; t < 32; t += 2) {
+                        const float x0 = __uint_as_float(a[t]), x1 = __uint_as_float(a[t + 1]);
+                        const float y0 = __uint_as_float(c[t]), y1 = __uint_as_float(c[t + 1]);
+                        s4[0] = fmaf(x0, x0, s4[0]);
+                        s4[1] = fmaf(x1, x1, s4[1]);
+                        s4[2] = fmaf(y0, y0, s4[2]);
+                        s4[3] = fmaf(y1, y1, s4[3]);
+                    }
+                    ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+                    // exchange with warp q ^ 2, which holds the other column half of the row
+                    m->ss_x[b & 1][half][r] = ss;
                 }
-                // exchange with warp q ^ 2, which holds the other column half of the row
-                m->ss_x[b & 1][half][r] = ss;
-                mbar_arrive(&m->ss_bar[b & 1]);
-                if (!__all_sync(0xffffffffu, mbar_wait(&m->ss_bar[b & 1], (uint32_t)((b >> 1) & 1),
-                                                       abort_flag, tlimit))) {
-                    ok = false;
-                    break;
+                // all four warps of the group, once per block.  Block b's buffer is next
+                // written in block b + 2, after every warp has passed block b + 1's
+                // barrier and so has read block b's partial sums: two buffers suffice.
+                named_barrier(1, C::GROUP);
+                if (ok) {
+                    const float other = m->ss_x[b & 1][half ^ 1][r];
+                    const float tot = half == 0 ? ss + other : other + ss;
+                    scale = rsqrtf(tot * (1.0f / C::D) + 1e-6f);
                 }
-                const float other = m->ss_x[b & 1][half ^ 1][r];
-                const float tot = half == 0 ? ss + other : other + ss;
-                scale = rsqrtf(tot * (1.0f / C::D) + 1e-6f);
             }
+            if (!ok) continue;
             const int nv = min(C::BETA, seq_len - b * C::BETA);
             const int R = 64 * (int)cta + r;
             const int R0 = 64 * (int)cta + 32 * (q & 1);     // first row of this warp's box

@@ -31,7 +31,8 @@ Every schedule is checked for:
   * a TMEM load only of the intended block's accumulator, with all its MMAs complete;
   * no shared-memory write (TMA or store) to a buffer that an in-flight MMA reads;
   * the RMSNorm partial sums read only after their writer stored them, and never
-    overwritten before the partner lane read them;
+    overwritten before the partner lane read them (the four warps of group O meet at a
+    named barrier once per block, modelled as a barrier of four arrivals per block);
   * no deadlock, and nothing in flight once every agent has finished.
 
 Not modelled: the timeout / abort paths, TMEM allocation, the numerical content, the
@@ -116,7 +117,7 @@ class PairModel:
     names deliberate protocol mistakes, for checking that the model catches them.
     """
 
-    def __init__(self, nb, tail=False, init=False, rms=False, nq=2, nks=2, nkd=2, nv=3, npb=2,
+    def __init__(self, nb, tail=False, init=False, rms=False, nq=2, nks=2, nkd=2, nv=4, npb=1,
                  mutations=(), static_checks=True):
         self.nb, self.tail, self.init, self.rms = nb, tail and nb > 0, init, rms
         self.NQ, self.NKS, self.NKD, self.NV, self.NPB = nq, nks, nkd, nv, npb
@@ -149,10 +150,11 @@ class PairModel:
     def compiles(nq, nks, nkd, nv, npb):
         """The kernel's static_asserts on the ring depths (PairCfg in prefill_pair.cuh): a
         ring's slot of block x is tested free on the done barrier of block x, which must not
-        have been lapped when the producer tests it; and group KV's wait for the value tile
-        of a partial last block (one block before its dKV) is exact only if the slot's
-        previous load fed a dKV that group has seen complete."""
-        return nq <= NF and nks <= NF and nv <= NF and nkd <= NDK and npb <= NF and nv >= 2
+        have been lapped when the producer tests it (the value ring has a release ring of
+        its own, v_free, as deep as itself); and group KV's wait for the value tile of a
+        partial last block (one block before its dKV) is exact only if the slot's previous
+        load fed a dKV that group has seen complete."""
+        return nq <= NF and nks <= NF and nkd <= NDK and npb <= NF and nv >= 2
 
     # ------------------------------------------------------------------ set-up
     def _cta_bars(self, c):
@@ -175,7 +177,8 @@ class PairModel:
             "p_ready": ring("p_ready", self.NPB, G),
             "snap_ready": ring("snap_ready", self.NKS, G),
             "drain": Barrier(f"drain@{c}", 2),
-            "ss_bar": ring("ss_bar", 2, WARPS),
+            "v_free": ring("v_free", self.NV, 1),
+            "ss_sync": Barrier(f"ss_sync@{c}", WARPS),
         }
 
     # ------------------------------------------------------------------ primitives
@@ -264,11 +267,12 @@ class PairModel:
         B0, Bc = self.bars[0], self.bars[c]
         nb, NQ, NKS, NKD, NV = self.nb, self.NQ, self.NKS, self.NKD, self.NV
         jq = js = jd = jv = 0
-        # value slots are released by P V (o_done); the mutation releases them at dKV
+        # value slots are released once group O has seen P V complete (v_free); the
+        # mutation releases them when dKV completes
         if "v_release_on_dkv" in self.mut:
             v_ring, v_n = Bc["dkv_done"], NDK
         else:
-            v_ring, v_n = Bc["o_done"], NF
+            v_ring, v_n = Bc["v_free"], NV
 
         def freed(ring, nring, j, depth):
             x = j - depth
@@ -461,22 +465,27 @@ class PairModel:
         who = f"O{c}.{w}"
         B0, Bc = self.bars[0], self.bars[c]
         for b in range(self.nb):
+            if "v_free_early" in self.mut and w == 0:   # frees the value slot before P V is done
+                Bc["v_free"][b % self.NV].arrive(b // self.NV, who)
             if "o_after_f1" in self.mut:      # waits for F1_b instead of P_b V_b
                 yield ("wait", Bc["f1_done"][b % NF], b // NF)
             else:
                 yield ("wait", Bc["o_done"][b % NF], b // NF)
+            if w == 0 and "v_free_early" not in self.mut:   # P V of block b read its value slot
+                Bc["v_free"][b % self.NV].arrive(b // self.NV, who)
             self.tmem_ld(who, ("O", c, w), self.O[c][b % NF], ("o", b))
             self.arrive(who, c, B0["f1_free"][b % NF], b // NF)
             yield STEP
             if self.rms:   # exchange of the row's partial sum of squares with warp w ^ 2
-                prev = self.ssx[c][b & 1][w]
+                slot = 0 if "ss_one_buffer" in self.mut else b & 1
+                prev = self.ssx[c][slot][w]
                 if prev is not None and not prev[1]:
                     raise ProtocolError(f"{who}: overwrites its partial sum of block {prev[0]} "
                                         f"before warp {w ^ 2} read it")
-                self.ssx[c][b & 1][w] = [b, False]
-                Bc["ss_bar"][b & 1].arrive(b >> 1, who)
-                yield ("wait", Bc["ss_bar"][b & 1], b >> 1)
-                other = self.ssx[c][b & 1][w ^ 2]
+                self.ssx[c][slot][w] = [b, False]
+                Bc["ss_sync"].arrive(b, who)          # the group's named barrier, block b
+                yield ("wait", Bc["ss_sync"], b)
+                other = self.ssx[c][slot][w ^ 2]
                 if other is None or other[0] != b:
                     raise ProtocolError(f"{who}: reads the partial sum of warp {w ^ 2} for block "
                                         f"{None if other is None else other[0]}, wants {b}")

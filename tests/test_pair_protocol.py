@@ -36,7 +36,7 @@ def _depths(hi=4):
 
 def test_every_accepted_ring_depth():
     accepted = [d for d in _depths() if PairModel.compiles(*d)]
-    assert (2, 2, 2, 3, 2) in accepted            # the kernel's depths
+    assert (2, 2, 2, 4, 1) in accepted            # the kernel's depths
     for i, (nq, nks, nkd, nv, npb) in enumerate(accepted):
         for nb, seed in ((3, i), (7, i + 1)):
             PairModel(nb, tail=bool(seed & 1), init=bool(seed & 2), rms=bool(seed & 4), nq=nq,
@@ -54,17 +54,17 @@ def _first_violation(seeds=300, **kw):
 
 @pytest.mark.parametrize("depths,barrier", [
     (dict(nkd=NDK + 1), "dkv_done"),      # key-dim slots tested on a 2-deep dkv_done ring
-    (dict(nq=NF + 1), "f1_done"),         # query slots tested on the f1_done ring
+    (dict(nq=NF + 1, npb=2), "f1_done"),  # query slots tested on the f1_done ring
+    (dict(nks=NF + 1), "f1_done"),        # key-row slots tested on the f1_done ring
     (dict(nv=1), "full_v"),               # group KV's tail wait meets an open previous phase
 ])
 def test_rejected_ring_depths_do_fail(depths, barrier):
     """A ring deeper than the done-barrier ring its slots are released on: the producer's
-    test of a slot can meet a barrier already lapped by the block one ring further on.  And
+    test of a slot can meet a barrier already lapped by the block one ring further on (for
+    the query ring the model reaches that schedule with two P buffers; with one, group P's
+    wait for the previous P V holds F1 back far enough, but the bound does not rely on it).  And
     a one-slot value ring: group KV's wait for the partial last block's value tile starts
-    while the slot's previous phase is still open.  (For a 4-deep value ring on the 3-deep
-    o_done ring the bound is conservative: lapping there needs P V of the block before to
-    complete while the producer has not yet tested the slot, and the model finds no such
-    schedule.)"""
+    while the slot's previous phase is still open."""
     with pytest.raises(ValueError):
         PairModel(6, **depths)
     msg = _first_violation(nb=8, tail=True, static_checks=False, **depths)
@@ -88,6 +88,10 @@ MUTANTS = {
     "no_snap_slot_wait": (dict(nb=6), ("KS", "snap")),
     # value slots released when dKV completes, though P V still reads them
     "v_release_on_dkv": (dict(nb=6), ("V", "full_v", "dkv_done")),
+    # group O frees the value slot before it has seen P V complete
+    "v_free_early": (dict(nb=7), ("V", "v_free", "full_v")),
+    # one RMSNorm partial-sum buffer: a fast warp overwrites it before its partner read it
+    "ss_one_buffer": (dict(nb=6, rms=True), ("partial sum",)),
     # group O loads O_b once F1_b completes, before P_b V_b has added to it
     "o_after_f1": (dict(nb=4), ("tmO",)),
 }
