@@ -20,7 +20,7 @@
 // TMEM read before the next state update, and the whole state stays on chip
 // for the entire sequence.
 //
-// Warp roles (320 threads):
+// Warp roles (448 threads):
 //   warp 0      TMA producer: Q_b, K_b (D columns) and V_b (64 columns) into a
 //               ring of NST shared-memory stages.
 //   warp 1      TMEM owner and MMA issuer (lane 0 issues; the warp zeroes the
@@ -28,10 +28,12 @@
 //   warps 2..5  group P: S_b -> causal mask -> bf16 P_b, written back into
 //               the first BETA/2 columns of S_b's TMEM buffer, where the
 //               O_b = P_b V_b product reads it as its A operand.
-//   warps 6..9  group O: KV += dKV_b, bf16 snapshot of KV, O_b -> (RMSNorm) ->
-//               bf16 global store, final fp32 state -> global store.
+//   warps 6..9  group O: O_b -> (RMSNorm) -> bf16 global store.
+//   warps 10..13 group KV: KV += dKV_b, bf16 snapshot of KV, final fp32 state.
+// The state chain (group KV) and the output (group O) run on separate warps, so
+// the next snapshot never waits behind an output store or the RMSNorm exchange.
 // MMA issue order per block b: O_b = P_b V_b, dKV_b = K_b^T V_b,
-// O_b += Q_b snap(KV_{<b}), release of the stage, then S_{b+1}.
+// O_b += Q_b snap(KV_{<b}), release of the stage, then S_{b+2}.
 // Every wait is bounded (see mbar_wait); on a timeout the CTA records
 // DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -94,7 +96,7 @@ struct TcCfg {
     static constexpr int NST_FIT =
         (SMEM_LIMIT - 1024 - 2 * SNAP_BYTES - MISC) / STAGE;
     static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;
-    static_assert(NST >= 2, "shared memory budget");
+    static_assert(NST >= 3, "shared memory budget: S runs two blocks ahead");
     // Blocks ahead of the TMA ring whose tiles are prefetched into L2, so that a
     // stage load is served from L2 rather than waiting on HBM.
     static constexpr int PF = LA_PREFETCH_BLOCKS;
@@ -113,7 +115,7 @@ struct TcCfg {
     static constexpr int TMEM_COLS = 512;
     static_assert(TM_DKV + 128 <= TMEM_COLS, "TMEM budget");
     static constexpr int GROUP = 128;           // threads of one epilogue group
-    static constexpr int THREADS = 64 + 2 * GROUP;
+    static constexpr int THREADS = 64 + 3 * GROUP;
     static constexpr uint32_t ID_S = idesc_bf16_f32(BETA, BETA, 0, 0);
     static constexpr uint32_t ID_PV = idesc_bf16_f32(BETA, 64, 0, 1);
     static constexpr uint32_t ID_QKV = idesc_bf16_f32(BETA, 64, 0, 1);
@@ -131,7 +133,7 @@ struct TcMisc {
     uint64_t dkv_full[2];
     uint64_t dkv_free[2];
     uint64_t ss_full[2];
-    uint64_t p_ready;
+    uint64_t p_ready[2];     // P_b written over S_b in TMEM buffer b % 2
     uint64_t snap_ready[2];  // snapshot u of the state is in buffer u % 2
     uint64_t drain;
     uint32_t tmem_base;
@@ -182,7 +184,8 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             mbar_init(&m->dkv_free[i], C::GROUP);
             mbar_init(&m->ss_full[i], C::GROUP);
         }
-        mbar_init(&m->p_ready, C::GROUP);
+        mbar_init(&m->p_ready[0], C::GROUP);
+        mbar_init(&m->p_ready[1], C::GROUP);
         mbar_init(&m->snap_ready[0], C::GROUP);
         mbar_init(&m->snap_ready[1], C::GROUP);
         mbar_init(&m->drain, 1);
@@ -286,17 +289,20 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         };
 
         // Per block b: O_b = P_b V_b, dKV_b = K_b^T V_b, O_b += Q_b snap(KV_{<b}); the stage
-        // is released; then S_{b+1} = Q_{b+1} K_{b+1}^T.  S_{b+1} is issued last so that its
-        // tiles, loaded when stage b-1 was released, have had a whole block to arrive; the
-        // epilogue turns S_{b+1} into P_{b+1} while the tensor pipe drains block b.
+        // is released; then S_{b+2} = Q_{b+2} K_{b+2}^T.  The scores run two blocks ahead, so
+        // group P turns S_{b+1} into P_{b+1} during block b and P V never waits for it.
+        // S_{b+2} reuses S_b's buffer, which held P_b: P_b V_b precedes it in this thread's
+        // MMA order.
         bool ok = nb == 0 || stage_in(0);
+        if (ok && nb > 1) ok = stage_in(1);
         for (int b = 0; ok && b < nb; ++b) {
             const int st = b % C::NST;
             const uint32_t sa = stage_addr(st);
             const uint32_t sV = sa + 2 * C::DB * C::BOX;
             const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
             const uint32_t dKV = tmem + C::TM_DKV + 64 * (b & 1);
-            if (!wwait(&m->p_ready, (uint32_t)(b & 1))) {
+            // p_ready[b % 2] phase b / 2; its next phase needs S_{b+2}, issued below
+            if (!wwait(&m->p_ready[b & 1], (uint32_t)((b >> 1) & 1))) {
                 ok = false;
                 break;
             }
@@ -344,7 +350,7 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 mma_commit(&m->empty[st]);
             }
             __syncwarp();
-            if (b + 1 < nb && !stage_in(b + 1)) {
+            if (b + 2 < nb && !stage_in(b + 2)) {
                 ok = false;
                 break;
             }
@@ -389,54 +395,17 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&m->p_ready);
+            mbar_arrive(&m->p_ready[b & 1]);
         }
         if (!ok) fail();
-    } else {
+    } else if (warp < 10) {
         // ------------------------------------------------------------ group O
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const int r = BETA == 128 ? 32 * q + lane : 16 * q + lane;   // query row in the block
         const bool r_ok = BETA == 128 || lane < 16;
-        const int i = D == 128 ? 32 * q + lane : 16 * q + lane;      // state row
-        const bool i_ok = D == 128 || lane < 16;
         const size_t o_col = (size_t)h * D + 64 * vs;
-        float kv[64];                                              // KV[i][64 vs .. 64 vs + 63]
-#pragma unroll
-        for (int t = 0; t < 64; ++t) kv[t] = 0.f;
         bool ok = true;
-        // snapshot u of KV into buffer u % 2 (bf16, 128-byte swizzled rows), then signal it
-        auto write_snap = [&](int u) {
-            const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (u & 1);
-            if (i_ok) {
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const uint32_t chunk = (uint32_t)(t ^ (i & 7));
-                    st_shared_v4(sSnap + i * 128 + (chunk << 4), pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
-                                 pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
-                                 pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
-                                 pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&m->snap_ready[u & 1]);
-        };
-        if (p.state_in != nullptr) {  // KV starts at the sequence's initial state
-            if (i_ok) {
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    p.state_in + (((size_t)sid * p.H + h) * D + i) * D + 64 * vs);
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float4 x = src[t];
-                    kv[4 * t] = x.x;
-                    kv[4 * t + 1] = x.y;
-                    kv[4 * t + 2] = x.z;
-                    kv[4 * t + 3] = x.w;
-                }
-            }
-            write_snap(0);
-        }
-
         auto write_o = [&](int j) -> bool {  // read O_j out of TMEM, normalise, store
             if (!wwait(&m->o_full[j & 1], (uint32_t)((j >> 1) & 1))) return false;
             tc_fence_after();
@@ -484,39 +453,79 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             return true;
         };
 
+        for (int b = 0; ok && b < nb; ++b) ok = write_o(b);
+        if (!ok) fail();
+    } else {
+        // ------------------------------------------------------------ group KV
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int i = D == 128 ? 32 * q + lane : 16 * q + lane;      // state row
+        const bool i_ok = D == 128 || lane < 16;
+        float kv[64];                                              // KV[i][64 vs .. 64 vs + 63]
+#pragma unroll
+        for (int t = 0; t < 64; ++t) kv[t] = 0.f;
+        bool ok = true;
+        // snapshot u of KV into buffer u % 2 (bf16, 128-byte swizzled rows), then signal it
+        auto write_snap = [&](int u) {
+            const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (u & 1);
+            if (i_ok) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const uint32_t chunk = (uint32_t)(t ^ (i & 7));
+                    st_shared_v4(sSnap + i * 128 + (chunk << 4), pack_bf16x2(kv[8 * t + 0], kv[8 * t + 1]),
+                                 pack_bf16x2(kv[8 * t + 2], kv[8 * t + 3]),
+                                 pack_bf16x2(kv[8 * t + 4], kv[8 * t + 5]),
+                                 pack_bf16x2(kv[8 * t + 6], kv[8 * t + 7]));
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&m->snap_ready[u & 1]);
+        };
+        if (p.state_in != nullptr) {  // KV starts at the sequence's initial state
+            if (i_ok) {
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    p.state_in + (((size_t)sid * p.H + h) * D + i) * D + 64 * vs);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float4 x = src[t];
+                    kv[4 * t] = x.x;
+                    kv[4 * t + 1] = x.y;
+                    kv[4 * t + 2] = x.z;
+                    kv[4 * t + 3] = x.w;
+                }
+            }
+            write_snap(0);
+        }
+
         for (int b = 0; b < nb; ++b) {
-            // (1) KV += dKV_b; the bf16 snapshot of KV_{<b+1} for O_{b+1} += Q_{b+1} KV
+            // KV += dKV_b; the bf16 snapshot of KV_{<b+1} for O_{b+1} += Q_{b+1} KV.
+            // dkv_full[b % 2] phase b / 2; its next phase (dKV_{b+2}) needs dkv_free below
             if (!wwait(&m->dkv_full[b & 1], (uint32_t)((b >> 1) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             {
-                uint32_t a[32], c[32];
+                // one 32-column half at a time, to keep the state and one load in registers
+                uint32_t a[32];
                 const uint32_t tK = tmem + C::TM_DKV + 64 * (b & 1) + lane_base;
                 tmem_ld32(tK, a);
-                tmem_ld32(tK + 32, c);
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 32; ++t) kv[t] += __uint_as_float(a[t]);
+                tmem_ld32(tK + 32, a);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&m->dkv_free[b & 1]);
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    kv[t] += __uint_as_float(a[t]);
-                    kv[32 + t] += __uint_as_float(c[t]);
-                }
+                for (int t = 0; t < 32; ++t) kv[32 + t] += __uint_as_float(a[t]);
             }
             if (b + 1 < nb) {
                 // Buffer (b+1)&1 was last read by O_{b-1} += Q_{b-1} KV, which finished
                 // before dKV_b (MMAs complete in issue order), so it is free here.
                 write_snap(b + 1);
             }
-            // (2) the previous block's output
-            if (b >= 1 && !write_o(b - 1)) {
-                ok = false;
-                break;
-            }
         }
-        if (ok && nb > 0) ok = write_o(nb - 1);
         if (ok && p.state != nullptr && i_ok) {  // final state K^T V of the sequence, fp32
             float4 *dst = reinterpret_cast<float4 *>(p.state + (((size_t)sid * p.H + h) * D + i) * D +
                                                      64 * vs);
