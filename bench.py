@@ -752,11 +752,12 @@ def bench_configs(api, synth, torch, stream, dev, peaks, cpu: bool):
     res["f4_mixed_batch"] = {
         "workload": f"{n1} one-token sequences + {nc} chunks of {L} tokens, H={H}, D={D}, bf16, "
                     f"each from its own state (read and written in place)",
-        "one_prefill_launch_ms": spread(ms_mix),
+        "one_prefill_call_ms": spread(ms_mix),
         "decode_step_plus_prefill_ms": spread(ms_split),
         "clocks": clk,
-        "note": "the same work as one la_prefill launch, and as la_decode_step for the one-token "
-                "rows followed by la_prefill for the chunks (two launches)"}
+        "note": "the same work as one la_prefill call (which runs the one-token sequences through "
+                "the decode kernel, in place, and the chunks through the prefill kernel), and as "
+                "la_decode_step on gathered one-token rows followed by la_prefill for the chunks"}
     res["status"] = api.status_string(api.device_status(stream))
     return res
 

@@ -104,6 +104,13 @@ enum {
  *             overwritten, by the same threads.
  *   stream    cudaStream_t for the launch.
  *
+ * With LA_BF16, the sequences of exactly one token are one decode step each (the
+ * arithmetic of la_decode_step, from X_s or from 0): the call launches the decode
+ * kernel for them, reading and writing their rows of q, k, v, o and their state
+ * slices in place, and the prefill kernel for the other sequences, both on
+ * `stream`.  (A mixed batch of one-token requests and longer chunks, jvyan.cn
+ * article section 2, then needs one call and no gather.)
+ *
  * Returns LA_OK once the work is enqueued.
  */
 la_status la_prefill(const void *q, const void *k, const void *v, void *o,

@@ -215,6 +215,47 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B
     }
 
     if (flags & LA_BF16) {
+        // Sequences of one token are decode steps: they go to the decode kernel (reading
+        // their rows of the packed arrays in place), the rest to the prefill kernel.  A
+        // one-token sequence would otherwise hold a whole prefill CTA (pair) for one row.
+        la::OneTokenTable ot;
+        ot.identity = 0;
+        int n1 = 0;
+        if (seqs.varlen) {
+            int w = 0;
+            for (int r = 0; r < S; ++r) {
+                if (seqs.seq_len[r] == 1) {
+                    ot.row[n1] = seqs.seq_start[r];
+                    ot.sid[n1] = seqs.seq_id[r];
+                    ++n1;
+                } else {
+                    seqs.seq_start[w] = seqs.seq_start[r];
+                    seqs.seq_len[w] = seqs.seq_len[r];
+                    seqs.seq_id[w] = seqs.seq_id[r];
+                    ++w;
+                }
+            }
+            S = w;
+        } else if (N == 1) {
+            ot.identity = 1;
+            n1 = S;
+            S = 0;
+        }
+        if (n1 > 0) {
+            using bf = __nv_bfloat16;
+            const bf *qb = static_cast<const bf *>(q), *kb = static_cast<const bf *>(k),
+                     *vb = static_cast<const bf *>(v);
+            bf *ob = static_cast<bf *>(o);
+            float *ws = (want_state || read_state) ? state_ws : nullptr;
+            if (D == 128)
+                la::decode_rows_kernel<128, bf><<<(unsigned)(n1 * H), 256, 0, stream>>>(
+                    qb, kb, vb, ob, ws, H, read_state ? 1 : 0, want_state ? 1 : 0, rms, ot);
+            else
+                la::decode_rows_kernel<64, bf><<<(unsigned)(n1 * H), 256, 0, stream>>>(
+                    qb, kb, vb, ob, ws, H, read_state ? 1 : 0, want_state ? 1 : 0, rms, ot);
+            if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+        }
+        if (S == 0) return LA_OK;
         const long long Tm = T;
         if (beta == 128 && D == 128) {
             // paired-CTA kernel: each CTA of a pair loads half of the rows / columns

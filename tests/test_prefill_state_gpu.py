@@ -169,3 +169,37 @@ def test_mixed_batch_decode_and_prefill(dtype, beta, D):
     tol = 1e-5 if dtype == torch.float32 else 2e-2
     assert oracle.rel_l2(o[rows], od) <= tol
     assert oracle.rel_l2(st[ones], dstate) <= 1e-6
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("rmsnorm", [False, True], ids=["plain", "rmsnorm"])
+@pytest.mark.parametrize("mode", ["read", "write", "none"])
+def test_one_token_sequences_in_a_packed_call(D, rmsnorm, mode):
+    """bf16 one-token sequences inside a packed call (they run as decode steps): from an
+    initial state that stays untouched (read), from zero with the final state written (write),
+    or with no state at all (none); against the oracle's single run of every sequence."""
+    H = 3
+    lens = [1, 200, 1, 1, 0, 129, 1]
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    S = len(lens)
+    q, k, v = synth.qkv(cu[-1], H, D, seed=37, dtype=torch.bfloat16, device="cuda")
+    x = synth.initial_state(S, H, D, tokens=500, seed=37, device="cuda")
+    x_host = x.cpu().numpy()
+    kw = dict(beta=128, cu_seqlens=cu, rmsnorm=rmsnorm)
+    if mode == "read":
+        o = api.prefill(q, k, v, initial_state=x, **kw)
+        st = None
+    elif mode == "write":
+        o, st = api.prefill(q, k, v, return_state=True, **kw)
+    else:
+        o = api.prefill(q, k, v, **kw)
+        st = None
+    torch.cuda.synchronize()
+    assert api.device_status() == api.LA_OK
+    init = x_host if mode == "read" else None
+    ref_o, ref_s = oracle.recurrent(q, k, v, cu, rmsnorm=rmsnorm, initial_state=init)
+    assert oracle.max_rel_l2_per_head(o, ref_o, cu) <= 2e-2
+    if mode == "read":
+        assert np.array_equal(x.cpu().numpy(), x_host)        # read only
+    if st is not None:
+        assert _state_err(st.cpu().numpy(), ref_s) <= 1e-5
