@@ -20,11 +20,13 @@
 // TMEM read before the next state update, and the whole state stays on chip
 // for the entire sequence.
 //
-// Warp roles (448 threads):
+// Warp roles (480 threads):
 //   warp 0      TMA producer: Q_b, K_b (D columns) and V_b (64 columns) into a
 //               ring of NST shared-memory stages.
-//   warp 1      TMEM owner and MMA issuer (lane 0 issues; the warp zeroes the
-//               V rows past a sequence end before they enter K^T V).
+//   warp 1      TMEM owner and MMA issuer A: the scores S and the inter-block
+//               term Q_b snap(KV_{<b}) (lane 0 issues).
+//   warp 14     MMA issuer B: O_b = P_b V_b and dKV_b = K_b^T V_b (the warp first
+//               zeroes the V rows past a sequence end).
 //   warps 2..5  group P: S_b -> causal mask -> bf16 P_b, written back into
 //               the first BETA/2 columns of S_b's TMEM buffer, where the
 //               O_b = P_b V_b product reads it as its A operand.
@@ -32,8 +34,9 @@
 //   warps 10..13 group KV: KV += dKV_b, bf16 snapshot of KV, final fp32 state.
 // The state chain (group KV) and the output (group O) run on separate warps, so
 // the next snapshot never waits behind an output store or the RMSNorm exchange.
-// MMA issue order per block b: O_b = P_b V_b, dKV_b = K_b^T V_b,
-// O_b += Q_b snap(KV_{<b}), release of the stage, then S_{b+2}.
+// Per block b, issuer B: O_b = P_b V_b, dKV_b = K_b^T V_b; issuer A, once P_b V_b
+// has completed: O_b += Q_b snap(KV_{<b}), then S_{b+2}.  Each releases the stage
+// of block b after its last product that reads it.
 // Every wait is bounded (see mbar_wait); on a timeout the CTA records
 // DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -115,7 +118,8 @@ struct TcCfg {
     static constexpr int TMEM_COLS = 512;
     static_assert(TM_DKV + 128 <= TMEM_COLS, "TMEM budget");
     static constexpr int GROUP = 128;           // threads of one epilogue group
-    static constexpr int THREADS = 64 + 3 * GROUP;
+    static constexpr int THREADS = 64 + 3 * GROUP + 32;
+    static constexpr int WARP_B = 14;           // issuer of P V and dKV
     static constexpr uint32_t ID_S = idesc_bf16_f32(BETA, BETA, 0, 0);
     static constexpr uint32_t ID_PV = idesc_bf16_f32(BETA, 64, 0, 1);
     static constexpr uint32_t ID_QKV = idesc_bf16_f32(BETA, 64, 0, 1);
@@ -134,6 +138,7 @@ struct TcMisc {
     uint64_t dkv_free[2];
     uint64_t ss_full[2];
     uint64_t p_ready[2];     // P_b written over S_b in TMEM buffer b % 2
+    uint64_t pv_done[2];     // O_b = P_b V_b complete (issuer B -> issuer A)
     uint64_t snap_ready[2];  // snapshot u of the state is in buffer u % 2
     uint64_t drain;
     uint32_t tmem_base;
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(&m->full[s], 1);
-            mbar_init(&m->empty[s], 1);
+            mbar_init(&m->empty[s], 2);   // one commit from each issuer
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&m->s_full[i], 1);
@@ -186,9 +191,11 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         }
         mbar_init(&m->p_ready[0], C::GROUP);
         mbar_init(&m->p_ready[1], C::GROUP);
+        mbar_init(&m->pv_done[0], 1);
+        mbar_init(&m->pv_done[1], 1);
         mbar_init(&m->snap_ready[0], C::GROUP);
         mbar_init(&m->snap_ready[1], C::GROUP);
-        mbar_init(&m->drain, 1);
+        mbar_init(&m->drain, 2);   // one commit from each issuer
         m->abort_flag = 0;
         fence_mbarrier_init_cluster();
         tma_prefetch_desc(&p.tmap_q);
@@ -257,20 +264,11 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        bool any_issued = false;
 
-        // Wait for block j's tiles, zero the V rows past the sequence end, issue S_j.
+        // Wait for block j's tiles and issue S_j.
         auto stage_in = [&](int j) -> bool {
             const int st = j % C::NST;
             if (!wwait(&m->full[st], (uint32_t)((j / C::NST) & 1))) return false;
-            const int nv = min(BETA, seq_len - j * BETA);
-            if (nv < BETA) {
-                const uint32_t v0 = stage_addr(st) + 2 * C::DB * C::BOX;
-                for (uint32_t a = v0 + nv * 128 + lane * 16; a < v0 + C::BOX; a += 32 * 16)
-                    st_shared_v4(a, 0u, 0u, 0u, 0u);
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t sa = stage_addr(st);
@@ -283,59 +281,37 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 }
                 mma_commit(&m->s_full[j & 1]);
             }
-            any_issued = true;
             __syncwarp();
             return true;
         };
 
-        // Per block b: O_b = P_b V_b, dKV_b = K_b^T V_b, O_b += Q_b snap(KV_{<b}); the stage
-        // is released; then S_{b+2} = Q_{b+2} K_{b+2}^T.  The scores run two blocks ahead, so
-        // group P turns S_{b+1} into P_{b+1} during block b and P V never waits for it.
-        // S_{b+2} reuses S_b's buffer, which held P_b: P_b V_b precedes it in this thread's
-        // MMA order.
+        // Per block b (issuer A): once issuer B's O_b = P_b V_b has completed, O_b +=
+        // Q_b snap(KV_{<b}); the stage's use by A is released; then S_{b+2} = Q_{b+2} K_{b+2}^T
+        // into S_b's buffer, whose P_b that P V has read.  The scores run two blocks ahead,
+        // so group P turns S_{b+1} into P_{b+1} during block b.
         bool ok = nb == 0 || stage_in(0);
         if (ok && nb > 1) ok = stage_in(1);
         for (int b = 0; ok && b < nb; ++b) {
             const int st = b % C::NST;
             const uint32_t sa = stage_addr(st);
-            const uint32_t sV = sa + 2 * C::DB * C::BOX;
             const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
-            const uint32_t dKV = tmem + C::TM_DKV + 64 * (b & 1);
-            // p_ready[b % 2] phase b / 2; its next phase needs S_{b+2}, issued below
-            if (!wwait(&m->p_ready[b & 1], (uint32_t)((b >> 1) & 1))) {
-                ok = false;
-                break;
+            if (b >= u0) {
+                // Snapshot b, the (b - u0)/2-th use of buffer b % 2.  Its next phase needs
+                // dKV_{b+1}, which issuer B issues only after o_full(b), committed below.
+                if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
+                    ok = false;
+                    break;
+                }
             }
-            if (b >= 2 && (!wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)) ||
-                           !wwait(&m->dkv_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)))) {
+            // pv_done[b % 2] phase b / 2; its next phase needs P_{b+2} V_{b+2}, which needs
+            // o_free after group O loaded O_b, after o_full(b) below
+            if (!wwait(&m->pv_done[b & 1], (uint32_t)((b >> 1) & 1))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             if (lane == 0) {
-                // O_b = P_b V_b, P_b from TMEM: 16 keys = 8 packed columns per K-step
-                const uint32_t tP = tmem + C::TM_S + BETA * (b & 1);
-                const uint64_t vd = desc_mnmajor_sw128(sV, C::BOX);
-                const uint64_t ktd = desc_mnmajor_sw128(sa + C::DB * C::BOX, C::BOX);
-#pragma unroll
-                for (int ks = 0; ks < BETA / 16; ++ks)
-                    mma_bf16_ts(dO, tP + 8 * ks, desc_add(vd, ks * 2048), C::ID_PV, ks > 0 ? 1u : 0u);
-#pragma unroll
-                for (int ks = 0; ks < BETA / 16; ++ks)  // dKV_b = K_b^T V_b
-                    mma_bf16_ss(dKV, desc_add(ktd, ks * 2048), desc_add(vd, ks * 2048), C::ID_KV,
-                                ks > 0 ? 1u : 0u);
-                mma_commit(&m->dkv_full[b & 1]);
-            }
-            __syncwarp();
-            if (b >= u0) {
-                // Snapshot b, the (b - u0)/2-th use of buffer b % 2.  One barrier per buffer:
-                // its next phase needs dKV_{b+1}, which this thread has not issued yet.
-                if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {  // O_b += Q_b snap(KV_{<b})
+                if (b >= u0) {  // O_b += Q_b snap(KV_{<b})
                     const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (b & 1);
                     const uint64_t qd = desc_kmajor_sw128(sa), sd = desc_mnmajor_sw128(sSnap, C::BOX);
 #pragma unroll
@@ -343,9 +319,6 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                         mma_bf16_ss(dO, desc_add(qd, (uint32_t)((ks >> 2) * C::BOX + (ks & 3) * 32)),
                                     desc_add(sd, ks * 2048), C::ID_QKV, 1u);
                 }
-                __syncwarp();
-            }
-            if (lane == 0) {
                 mma_commit(&m->o_full[b & 1]);
                 mma_commit(&m->empty[st]);
             }
@@ -356,7 +329,73 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             }
         }
         if (!ok) fail();
-        if (any_issued && lane == 0) {  // every issued MMA has finished before TMEM is freed
+        if (nb > 0 && lane == 0) {  // every issued MMA has finished before TMEM is freed
+            mma_commit(&m->drain);
+            mbar_wait(&m->drain, 0u, nullptr, tlimit);
+        }
+        __syncwarp();
+    } else if (warp == C::WARP_B) {
+        // ------------------------------------------------------------ MMA issuer B
+        // Per block b: O_b = P_b V_b (initialising O_b), then dKV_b = K_b^T V_b.  The value
+        // rows past a sequence end are zeroed first (no product before them reads V_b).
+        bool ok = true;
+        for (int b = 0; b < nb; ++b) {
+            const int st = b % C::NST;
+            const uint32_t sa = stage_addr(st);
+            const uint32_t sV = sa + 2 * C::DB * C::BOX;
+            const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
+            const uint32_t dKV = tmem + C::TM_DKV + 64 * (b & 1);
+            // full[st] phase b / NST: its next phase needs both issuers' release of block b;
+            // p_ready[b % 2] phase b / 2: its next phase needs S_{b+2}, which issuer A issues
+            // only after this P V; o_free: group O has loaded O_{b-2} from this buffer
+            if (!wwait(&m->full[st], (uint32_t)((b / C::NST) & 1)) ||
+                !wwait(&m->p_ready[b & 1], (uint32_t)((b >> 1) & 1)) ||
+                (b >= 2 && !wwait(&m->o_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)))) {
+                ok = false;
+                break;
+            }
+            const int nv = min(BETA, seq_len - b * BETA);
+            if (nv < BETA) {
+                for (uint32_t a = sV + nv * 128 + lane * 16; a < sV + C::BOX; a += 32 * 16)
+                    st_shared_v4(a, 0u, 0u, 0u, 0u);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            tc_fence_after();
+            if (lane == 0) {
+                // O_b = P_b V_b, P_b from TMEM: 16 keys = 8 packed columns per K-step
+                const uint32_t tP = tmem + C::TM_S + BETA * (b & 1);
+                const uint64_t vd = desc_mnmajor_sw128(sV, C::BOX);
+#pragma unroll
+                for (int ks = 0; ks < BETA / 16; ++ks)
+                    mma_bf16_ts(dO, tP + 8 * ks, desc_add(vd, ks * 2048), C::ID_PV, ks > 0 ? 1u : 0u);
+                mma_commit(&m->pv_done[b & 1]);
+            }
+            __syncwarp();
+            // dKV_b feeds snapshot b + 1, which group KV writes into the buffer of snapshot
+            // b - 1: Q_{b-1} snap_{b-1} (issuer A) must have completed (o_full(b-1); its next
+            // phase needs P_{b+1} V_{b+1}, issued later here).  dkv_free: group KV has loaded
+            // dKV_{b-2} from this buffer.
+            if ((b >= 1 && !wwait(&m->o_full[(b - 1) & 1], (uint32_t)(((b - 1) >> 1) & 1))) ||
+                (b >= 2 && !wwait(&m->dkv_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t vd = desc_mnmajor_sw128(sV, C::BOX);
+                const uint64_t ktd = desc_mnmajor_sw128(sa + C::DB * C::BOX, C::BOX);
+#pragma unroll
+                for (int ks = 0; ks < BETA / 16; ++ks)
+                    mma_bf16_ss(dKV, desc_add(ktd, ks * 2048), desc_add(vd, ks * 2048), C::ID_KV,
+                                ks > 0 ? 1u : 0u);
+                mma_commit(&m->dkv_full[b & 1]);
+                mma_commit(&m->empty[st]);
+            }
+            __syncwarp();
+        }
+        if (!ok) fail();
+        if (nb > 0 && lane == 0) {  // every issued MMA has finished before TMEM is freed
             mma_commit(&m->drain);
             mbar_wait(&m->drain, 0u, nullptr, tlimit);
         }
@@ -365,7 +404,8 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         // ------------------------------------------------------------ group P
         // S_b and P_b share a TMEM buffer: chunk cc reads S columns [64cc, 64cc+64)
         // and writes P columns [32cc, 32cc+32), which lie in S columns already read.
-        // S_{b+2} reuses the buffer only after O_b = P_b V_b, in MMA issue order.
+        // Issuer A issues S_{b+2} into the buffer only after it has seen O_b = P_b V_b
+        // (issuer B) complete.
         const int q = warp & 3;                    // TMEM lane quadrant of this warp
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const int r = BETA == 128 ? 32 * q + lane : 16 * q + lane;   // query row in the block
@@ -455,7 +495,7 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
 
         for (int b = 0; ok && b < nb; ++b) ok = write_o(b);
         if (!ok) fail();
-    } else {
+    } else if (warp < C::WARP_B) {
         // ------------------------------------------------------------ group KV
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
