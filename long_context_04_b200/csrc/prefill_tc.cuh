@@ -23,10 +23,10 @@
 // Warp roles (480 threads):
 //   warp 0      TMA producer: Q_b, K_b (D columns) and V_b (64 columns) into a
 //               ring of NST shared-memory stages.
-//   warp 1      TMEM owner and MMA issuer A: the scores S and the inter-block
-//               term Q_b snap(KV_{<b}) (lane 0 issues).
-//   warp 14     MMA issuer B: O_b = P_b V_b and dKV_b = K_b^T V_b (the warp first
-//               zeroes the V rows past a sequence end).
+//   warp 1      TMEM owner and MMA issuer A: the scores S and dKV_b = K_b^T V_b
+//               (lane 0 issues).
+//   warp 14     MMA issuer B: O_b = P_b V_b and the inter-block term Q_b snap(KV_{<b})
+//               (the warp first zeroes the V rows past a sequence end).
 //   warps 2..5  group P: S_b -> causal mask -> bf16 P_b, written back into
 //               the first BETA/2 columns of S_b's TMEM buffer, where the
 //               O_b = P_b V_b product reads it as its A operand.
@@ -34,9 +34,10 @@
 //   warps 10..13 group KV: KV += dKV_b, bf16 snapshot of KV, final fp32 state.
 // The state chain (group KV) and the output (group O) run on separate warps, so
 // the next snapshot never waits behind an output store or the RMSNorm exchange.
-// Per block b, issuer B: O_b = P_b V_b, dKV_b = K_b^T V_b; issuer A, once P_b V_b
-// has completed: O_b += Q_b snap(KV_{<b}), then S_{b+2}.  Each releases the stage
-// of block b after its last product that reads it.
+// Per block b, issuer B: O_b = P_b V_b, then O_b += Q_b snap(KV_{<b}) on the same
+// accumulator; issuer A, once P_b V_b has completed: dKV_b, then S_{b+2}.  Each
+// issues 12 of the 24 MMAs of a block (at beta = 64) and releases the stage of
+// block b after its last product that reads it.
 // Every wait is bounded (see mbar_wait); on a timeout the CTA records
 // DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -138,7 +139,8 @@ struct TcMisc {
     uint64_t dkv_free[2];
     uint64_t ss_full[2];
     uint64_t p_ready[2];     // P_b written over S_b in TMEM buffer b % 2
-    uint64_t pv_done[2];     // O_b = P_b V_b complete (issuer B -> issuer A)
+    uint64_t pv_done[2];     // P_b V_b complete (issuer B -> issuer A)
+    uint64_t tail_zeroed;    // issuer B zeroed the value rows past the sequence end
     uint64_t snap_ready[2];  // snapshot u of the state is in buffer u % 2
     uint64_t drain;
     uint32_t tmem_base;
@@ -193,6 +195,7 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         mbar_init(&m->p_ready[1], C::GROUP);
         mbar_init(&m->pv_done[0], 1);
         mbar_init(&m->pv_done[1], 1);
+        mbar_init(&m->tail_zeroed, 1);
         mbar_init(&m->snap_ready[0], C::GROUP);
         mbar_init(&m->snap_ready[1], C::GROUP);
         mbar_init(&m->drain, 2);   // one commit from each issuer
@@ -285,41 +288,41 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
             return true;
         };
 
-        // Per block b (issuer A): once issuer B's O_b = P_b V_b has completed, O_b +=
-        // Q_b snap(KV_{<b}); the stage's use by A is released; then S_{b+2} = Q_{b+2} K_{b+2}^T
-        // into S_b's buffer, whose P_b that P V has read.  The scores run two blocks ahead,
-        // so group P turns S_{b+1} into P_{b+1} during block b.
+        // Per block b (issuer A): once issuer B's P_b V_b has completed, dKV_b = K_b^T V_b;
+        // the stage's use by A is released; then S_{b+2} = Q_{b+2} K_{b+2}^T into S_b's
+        // buffer, whose P_b that P V has read.  The scores run two blocks ahead, so group P
+        // turns S_{b+1} into P_{b+1} during block b.  P_b V_b completing also means that
+        // issuer B zeroed the value rows past a sequence end (before P V) and that its
+        // Q_{b-1} snap_{b-1} has completed (issued before P V): group KV then writes snapshot
+        // b + 1 into that snapshot's buffer once dKV_b is done.
         bool ok = nb == 0 || stage_in(0);
         if (ok && nb > 1) ok = stage_in(1);
         for (int b = 0; ok && b < nb; ++b) {
             const int st = b % C::NST;
             const uint32_t sa = stage_addr(st);
-            const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
-            if (b >= u0) {
-                // Snapshot b, the (b - u0)/2-th use of buffer b % 2.  Its next phase needs
-                // dKV_{b+1}, which issuer B issues only after o_full(b), committed below.
-                if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
-                    ok = false;
-                    break;
-                }
-            }
-            // pv_done[b % 2] phase b / 2; its next phase needs P_{b+2} V_{b+2}, which needs
-            // o_free after group O loaded O_b, after o_full(b) below
-            if (!wwait(&m->pv_done[b & 1], (uint32_t)((b >> 1) & 1))) {
+            const uint32_t sV = sa + 2 * C::DB * C::BOX;
+            const uint32_t dKV = tmem + C::TM_DKV + 64 * (b & 1);
+            // pv_done[b % 2] phase b / 2: its next phase needs P_{b+2} V_{b+2}, issued after
+            // Q_{b+1} snap_{b+1}, which waits for snapshot b + 1 from the dKV_b below.
+            // dkv_free: group KV has loaded dKV_{b-2} from this buffer.
+            // tail_zeroed (single phase): issuer B's zeroed value rows, published with a
+            // release arrival, before dKV of a partial last block reads them
+            const bool last_tail = b == nb - 1 && seq_len < nb * BETA;
+            if (!wwait(&m->pv_done[b & 1], (uint32_t)((b >> 1) & 1)) ||
+                (b >= 2 && !wwait(&m->dkv_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1))) ||
+                (last_tail && !wwait(&m->tail_zeroed, 0u))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             if (lane == 0) {
-                if (b >= u0) {  // O_b += Q_b snap(KV_{<b})
-                    const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (b & 1);
-                    const uint64_t qd = desc_kmajor_sw128(sa), sd = desc_mnmajor_sw128(sSnap, C::BOX);
+                const uint64_t vd = desc_mnmajor_sw128(sV, C::BOX);
+                const uint64_t ktd = desc_mnmajor_sw128(sa + C::DB * C::BOX, C::BOX);
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        mma_bf16_ss(dO, desc_add(qd, (uint32_t)((ks >> 2) * C::BOX + (ks & 3) * 32)),
-                                    desc_add(sd, ks * 2048), C::ID_QKV, 1u);
-                }
-                mma_commit(&m->o_full[b & 1]);
+                for (int ks = 0; ks < BETA / 16; ++ks)
+                    mma_bf16_ss(dKV, desc_add(ktd, ks * 2048), desc_add(vd, ks * 2048), C::ID_KV,
+                                ks > 0 ? 1u : 0u);
+                mma_commit(&m->dkv_full[b & 1]);
                 mma_commit(&m->empty[st]);
             }
             __syncwarp();
@@ -336,15 +339,15 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
         __syncwarp();
     } else if (warp == C::WARP_B) {
         // ------------------------------------------------------------ MMA issuer B
-        // Per block b: O_b = P_b V_b (initialising O_b), then dKV_b = K_b^T V_b.  The value
-        // rows past a sequence end are zeroed first (no product before them reads V_b).
+        // Per block b: O_b = P_b V_b (initialising O_b), then, in order on the same
+        // accumulator, O_b += Q_b snap(KV_{<b}).  The value rows past a sequence end are
+        // zeroed first (no product before them reads V_b).
         bool ok = true;
         for (int b = 0; b < nb; ++b) {
             const int st = b % C::NST;
             const uint32_t sa = stage_addr(st);
             const uint32_t sV = sa + 2 * C::DB * C::BOX;
             const uint32_t dO = tmem + C::TM_O + 64 * (b & 1);
-            const uint32_t dKV = tmem + C::TM_DKV + 64 * (b & 1);
             // full[st] phase b / NST: its next phase needs both issuers' release of block b;
             // p_ready[b % 2] phase b / 2: its next phase needs S_{b+2}, which issuer A issues
             // only after this P V; o_free: group O has loaded O_{b-2} from this buffer
@@ -359,6 +362,8 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 for (uint32_t a = sV + nv * 128 + lane * 16; a < sV + C::BOX; a += 32 * 16)
                     st_shared_v4(a, 0u, 0u, 0u, 0u);
                 fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&m->tail_zeroed);   // for issuer A's dKV
             }
             __syncwarp();
             tc_fence_after();
@@ -372,24 +377,27 @@ __global__ void __launch_bounds__(TcCfg<BETA, D>::THREADS, 1)
                 mma_commit(&m->pv_done[b & 1]);
             }
             __syncwarp();
-            // dKV_b feeds snapshot b + 1, which group KV writes into the buffer of snapshot
-            // b - 1: Q_{b-1} snap_{b-1} (issuer A) must have completed (o_full(b-1); its next
-            // phase needs P_{b+1} V_{b+1}, issued later here).  dkv_free: group KV has loaded
-            // dKV_{b-2} from this buffer.
-            if ((b >= 1 && !wwait(&m->o_full[(b - 1) & 1], (uint32_t)(((b - 1) >> 1) & 1))) ||
-                (b >= 2 && !wwait(&m->dkv_free[b & 1], (uint32_t)(((b - 2) >> 1) & 1)))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t vd = desc_mnmajor_sw128(sV, C::BOX);
-                const uint64_t ktd = desc_mnmajor_sw128(sa + C::DB * C::BOX, C::BOX);
+            if (b >= u0) {
+                // Snapshot b, the (b - u0)/2-th use of buffer b % 2.  Its next phase needs
+                // dKV_{b+1}, which issuer A issues only after P_{b+1} V_{b+1}, issued here
+                // after this product.
+                if (!wwait(&m->snap_ready[b & 1], (uint32_t)(((b - u0) >> 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {  // O_b += Q_b snap(KV_{<b})
+                    const uint32_t sSnap = sbase + C::OFF_SNAP + C::SNAP_BYTES * (b & 1);
+                    const uint64_t qd = desc_kmajor_sw128(sa), sd = desc_mnmajor_sw128(sSnap, C::BOX);
 #pragma unroll
-                for (int ks = 0; ks < BETA / 16; ++ks)
-                    mma_bf16_ss(dKV, desc_add(ktd, ks * 2048), desc_add(vd, ks * 2048), C::ID_KV,
-                                ks > 0 ? 1u : 0u);
-                mma_commit(&m->dkv_full[b & 1]);
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        mma_bf16_ss(dO, desc_add(qd, (uint32_t)((ks >> 2) * C::BOX + (ks & 3) * 32)),
+                                    desc_add(sd, ks * 2048), C::ID_QKV, 1u);
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {
+                mma_commit(&m->o_full[b & 1]);
                 mma_commit(&m->empty[st]);
             }
             __syncwarp();

@@ -7,10 +7,10 @@ mbarriers that order them.  Each agent is a generator mirroring one role of the 
 kernel's order, one step per wait, arrival, TMA issue, store or MMA issue:
 
     producer<c>        warp 0: Q, K and the value slice of every block into a ring of stages
-    A<c>               issuer A: the scores S_b (two blocks ahead) and the inter-block term
-                       O_b += Q_b snap_b, once issuer B's O_b = P_b V_b has completed
-    B<c>               issuer B: O_b = P_b V_b and dKV_b = K_b^T V_b (it zeroes the value rows
-                       past the sequence end first)
+    A<c>               issuer A: the scores S_b (two blocks ahead) and dKV_b = K_b^T V_b,
+                       once issuer B's O_b = P_b V_b has completed
+    B<c>               issuer B: O_b = P_b V_b (it zeroes the value rows past the sequence
+                       end first), then O_b += Q_b snap_b on the same accumulator
     P<c>.<w>, O<c>.<w>, KV<c>.<w>
                        warp w (0..3) of group P (S -> P in TMEM), group O (O -> RMSNorm ->
                        store) and group KV (state, snapshots) of CTA c
@@ -118,6 +118,7 @@ class TcModel:
             "snap_ready": ring("snap_ready", 2, WARPS),
             "ss_full": ring("ss_full", 2, WARPS),
             "drain": Barrier(f"drain@{c}", 2),
+            "tail_zeroed": Barrier(f"tail_zeroed@{c}", 1),
         }
 
     # ------------------------------------------------------------------ primitives
@@ -205,6 +206,9 @@ class TcModel:
             yield ("wait", B["full"][b % NST], b // NST)
 
     def issuer_a(self, c):
+        """The scores (two blocks ahead) and dKV_b, once P_b V_b has completed: issuer B zeroes
+        the tail rows before it, and issues Q_{b-1} snap_{b-1} before it (so group KV may write
+        snapshot b + 1 into that snapshot's buffer once dKV_b is done)."""
         who, B, NST, nb = f"A{c}", self.bars[c], self.NST, self.nb
 
         def stage_in(j):
@@ -221,17 +225,18 @@ class TcModel:
             yield from stage_in(1)
         for b in range(nb):
             st = b % NST
-            if b >= self.u0:
-                u = b if "snap_one_buffer" not in self.mut else 0
-                yield ("wait", B["snap_ready"][u & 1], (b - self.u0) >> 1
-                       if "snap_one_buffer" not in self.mut else b - self.u0)
+            last_tail = self.tail and b == nb - 1
             if "a_no_pv_done_wait" not in self.mut:
                 yield ("wait", B["pv_done"][b & 1], b >> 1)
-            if b >= self.u0:
-                sbuf = self.SNAP[c][0 if "snap_one_buffer" in self.mut else b & 1]
-                self.mma(who, f"QKV_{b}", [(self.Q[c][st], ("q", b)), (sbuf, ("snap", b))],
-                         [(self.O[c][b & 1], ("o_pv", b), True, ("o", b))])
-            self.commit(who, B["o_full"][b & 1], b >> 1)
+            if b >= 2:
+                yield ("wait", B["dkv_free"][b & 1], (b - 2) >> 1)
+            if last_tail:
+                yield ("wait", B["tail_zeroed"], 0)
+            vbuf = self.V[c][st]
+            self.mma(who, f"dKV_{b}", [(self.K[c][st], ("k", b)), (vbuf, ("v", b))],
+                     [(self.DKV[c][b & 1], None, False, ("dkv", b))],
+                     zeroed=[vbuf] if last_tail else [])
+            self.commit(who, B["dkv_full"][b & 1], b >> 1)
             self.commit(who, B["empty"][st], b // NST)
             yield STEP
             if b + 2 < nb:
@@ -240,7 +245,10 @@ class TcModel:
         yield ("wait", B["drain"], 0)
 
     def issuer_b(self, c):
+        """P_b V_b (zeroing the tail rows first), then, in order on the same accumulator,
+        O_b += Q_b snap_b."""
         who, B, NST, nb = f"B{c}", self.bars[c], self.NST, self.nb
+        qkv_first = "b_qkv_first" in self.mut
         for b in range(nb):
             st = b % NST
             yield ("wait", B["full"][st], b // NST)
@@ -252,8 +260,13 @@ class TcModel:
                 yield ("wait", B["o_free"][b & 1], (b - 2) >> 1)
             last_tail = self.tail and b == nb - 1
             vbuf = self.V[c][st]
+            if qkv_first and b >= self.u0:     # the inter-block term issued before P V
+                yield ("wait", B["snap_ready"][b & 1], (b - self.u0) >> 1)
+                self.mma(who, f"QKV_{b}", [(self.Q[c][st], ("q", b)), (self.SNAP[c][b & 1], ("snap", b))],
+                         [(self.O[c][b & 1], ("o_pv", b), True, ("o", b))])
             if last_tail and "zero_after_pv" not in self.mut:
                 self._zero(who, vbuf, ("v", b))
+                B["tail_zeroed"].arrive(0, who)
             self.mma(who, f"PV_{b}", [(self.SQ[c][b & 1][w], ("P", b)) for w in range(WARPS)] +
                      [(vbuf, ("v", b))], [(self.O[c][b & 1], None, False, ("o_pv", b))],
                      zeroed=[vbuf] if last_tail else [])
@@ -261,14 +274,15 @@ class TcModel:
             yield STEP
             if last_tail and "zero_after_pv" in self.mut:
                 self._zero(who, vbuf, ("v", b))
-            if b >= 1 and "b_no_o_full_wait" not in self.mut:
-                yield ("wait", B["o_full"][(b - 1) & 1], (b - 1) >> 1)
-            if b >= 2:
-                yield ("wait", B["dkv_free"][b & 1], (b - 2) >> 1)
-            self.mma(who, f"dKV_{b}", [(self.K[c][st], ("k", b)), (vbuf, ("v", b))],
-                     [(self.DKV[c][b & 1], None, False, ("dkv", b))],
-                     zeroed=[vbuf] if last_tail else [])
-            self.commit(who, B["dkv_full"][b & 1], b >> 1)
+                B["tail_zeroed"].arrive(0, who)
+            if b >= self.u0 and not qkv_first:
+                one = "snap_one_buffer" in self.mut
+                yield ("wait", B["snap_ready"][0 if one else b & 1],
+                       (b - self.u0) if one else (b - self.u0) >> 1)
+                sbuf = self.SNAP[c][0 if one else b & 1]
+                self.mma(who, f"QKV_{b}", [(self.Q[c][st], ("q", b)), (sbuf, ("snap", b))],
+                         [(self.O[c][b & 1], ("o_pv", b), True, ("o", b))])
+            self.commit(who, B["o_full"][b & 1], b >> 1)
             if "single_empty_arrival" not in self.mut:
                 self.commit(who, B["empty"][st], b // NST)
             yield STEP

@@ -56,15 +56,16 @@ def test_two_stages_still_safe():
 
 # mutation -> (shape, words of which the first violation must name one)
 MUTANTS = {
-    # issuer A adds the inter-block term / writes S_{b+2} without waiting for P_b V_b
-    "a_no_pv_done_wait": (dict(nb=6, init=True), ("another issuer", "tmO", "tmS")),
-    # issuer B issues dKV_b before Q_{b-1} snap_{b-1} completed: group KV then writes
-    # snapshot b + 1 into a buffer that product still reads
-    "b_no_o_full_wait": (dict(nb=8, init=True), ("snap",)),
+    # issuer A issues dKV_b and S_{b+2} without waiting for P_b V_b: dKV_b may read the value
+    # tile before issuer B zeroed its tail rows, S_{b+2} may overwrite P_b under P V, and
+    # group KV may write snapshot b + 1 over snapshot b - 1 before Q_{b-1} snap_{b-1} read it
+    "a_no_pv_done_wait": (dict(nb=6, tail=True), ("another issuer", "tmS", "zeroed", "snap")),
+    # issuer B adds the inter-block term before P V, which initialises the accumulator
+    "b_qkv_first": (dict(nb=5, init=True), ("tmO", "another issuer")),
     # issuer B's P V overwrites O before group O loaded it
     "b_no_o_free_wait": (dict(nb=7), ("tmO",)),
-    # only issuer A releases a stage: the producer reloads it under issuer B's dKV
-    "single_empty_arrival": (dict(nb=9), ("TMA", "K", "V")),
+    # only issuer A releases a stage: the producer reloads it under issuer B's products
+    "single_empty_arrival": (dict(nb=9, init=True), ("TMA", "Q", "V")),
     # one P-ready barrier instead of a ring of two: with the scores two blocks ahead, group P
     # can complete the next phase before issuer B waits on this one
     "p_ready_single": (dict(nb=8), ("p_ready",)),
